@@ -1,0 +1,368 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU).
+
+Each test checks the oracle against something the pages or mathematics fix: a
+hand-derived worked example (tests/golden), a closed form, an invariant, a
+library routine, or brute force on tiny inputs. They are chosen so that a
+dropped term, a wrong sign or index, a transposed operand, or a swapped
+gate/up would fail at least one of them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from conftest import read_golden
+from synth import FFNWeights, QWeight, FMT_INT4_G32, FMT_INT8_ROW
+
+pytestmark = pytest.mark.cpu
+
+
+def _hex16(tokens, dtype):
+    return np.array([int(t, 16) for t in tokens], dtype=np.uint16).view(dtype)
+
+
+# --------------------------------------------------------------------------- dequant
+
+
+def test_dequant_int4_golden_block():
+    kv, _ = read_golden("int4_affine_g32_block.txt")
+    packed = np.array([int(t, 16) for t in kv["packed_hex"]], np.uint8)[None, :]
+    scale = _hex16(kv["scale_fp16_hex"], np.float16)[None, :]
+    mn = _hex16(kv["min_fp16_hex"], np.float16)[None, :]
+    want = np.array([float(t) for t in kv["expected"]])
+    got = oracle.dequant_int4_affine_g32(packed, scale, mn)[0]
+    assert np.array_equal(got, want)
+    # The fp32 form is exact: rounding to fp32 changes nothing.
+    assert np.array_equal(oracle.f32(got), want)
+
+
+def test_dequant_int4_subnormal_scale_exact():
+    kv, _ = read_golden("int4_affine_g32_subnormal.txt")
+    packed = np.array([int(t, 16) for t in kv["packed_hex"]], np.uint8)[None, :]
+    scale = _hex16(kv["scale_fp16_hex"], np.float16)[None, :]
+    mn = _hex16(kv["min_fp16_hex"], np.float16)[None, :]
+    want = np.array([float(t) for t in kv["expected"]])
+    assert np.array_equal(oracle.dequant_int4_affine_g32(packed, scale, mn)[0], want)
+
+
+def test_dequant_int8_golden_block():
+    kv, _ = read_golden("int8_row_block.txt")
+    q = np.array([[int(t) for t in kv["q_row0"]], [int(t) for t in kv["q_row1"]]], np.int8)
+    scale = _hex16(kv["scale_fp16_hex"], np.float16)
+    got = oracle.dequant_int8_row(q, scale)
+    assert np.array_equal(got[0], [float(t) for t in kv["expected_row0"]])
+    assert np.array_equal(got[1], [float(t) for t in kv["expected_row1"]])
+
+
+def test_dequant_int4_fp32_exact_on_config_ranges():
+    """q*scale + min is exact in fp32 for the configurations' value ranges: the
+    fp32 evaluation with one fused step equals the float64 one."""
+    rng = np.random.default_rng(5)
+    w = synth.random_qweight(FMT_INT4_G32, 64, 256, rng)
+    ref = oracle.dequant(w)
+    q = oracle.int4_codes(w.q).astype(np.float32)
+    g = np.arange(256) // 32
+    s = w.scale.astype(np.float32)[:, g]
+    m = w.min.astype(np.float32)[:, g]
+    prod = (q.astype(np.float64) * s.astype(np.float64))
+    assert np.array_equal(oracle.f32(prod), prod)            # the product is exact in fp32
+    assert np.array_equal((np.float32(1) * (q * s) + m).astype(np.float64), ref)
+
+
+# --------------------------------------------------------------------------- rounding
+
+
+def test_bf16_rounding_golden():
+    _, rows = read_golden("bf16_rounding.txt")
+    vals = np.array([float(r[0]) for r in rows])
+    want = np.array([int(r[1], 16) for r in rows], np.uint16)
+    assert np.array_equal(oracle.bf16_bits(vals), want)
+
+
+def test_bf16_rounding_matches_torch_on_fp32_values():
+    rng = np.random.default_rng(0)
+    v = (rng.standard_normal(20000) * np.exp(rng.uniform(-30, 30, 20000))).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.bf16_bits(v.astype(np.float64)), ref)
+
+
+def test_activations_match_torch():
+    g = torch.linspace(-12, 12, 4001, dtype=torch.float64)
+    assert np.allclose(oracle.silu(g.numpy()), torch.nn.functional.silu(g).numpy(), rtol=1e-14, atol=1e-300)
+    assert np.allclose(oracle.gelu_tanh(g.numpy()),
+                       torch.nn.functional.gelu(g, approximate="tanh").numpy(), rtol=1e-13, atol=1e-15)
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    assert oracle.silu(np.array([64.0]))[0] == 64.0
+
+
+# --------------------------------------------------------------------------- helpers
+
+
+def _int8_matrix(values: np.ndarray, scale) -> QWeight:
+    """INT8 weights with integer entries and one per-row scale."""
+    N, K = values.shape
+    sc = np.full(N, scale, np.float16) if np.isscalar(scale) else np.asarray(scale, np.float16)
+    return QWeight(FMT_INT8_ROW, N, K, values.astype(np.int8), sc)
+
+
+def _int4_matrix(codes: np.ndarray, scale, mn) -> QWeight:
+    N, K = codes.shape
+    packed = (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+    s = np.full((N, K // 32), scale, np.float16)
+    m = np.full((N, K // 32), mn, np.float16)
+    return QWeight(FMT_INT4_G32, N, K, packed, s, m)
+
+
+def _perm_matrix(n, shift):
+    P = np.zeros((n, n), np.int64)
+    P[np.arange(n), (np.arange(n) + shift) % n] = 1      # (P x)[i] = x[i + shift]
+    return P
+
+
+# --------------------------------------------------------------------------- dense FFN
+
+
+@pytest.mark.parametrize("fmt", [FMT_INT8_ROW, FMT_INT4_G32])
+def test_dense_permutation_closed_form(fmt):
+    """gate = 2 P1, up = Q/2... with non-symmetric permutations: a transposed
+    operand, swapped gate/up or a dropped scale changes which entries meet."""
+    n, M = 64, 3
+    P1, P2, P3 = _perm_matrix(n, 5), _perm_matrix(n, 0), _perm_matrix(n, 17)
+    if fmt == FMT_INT8_ROW:
+        gate, up, down = _int8_matrix(P1, 2.0), _int8_matrix(P2, 0.5), _int8_matrix(P3, 1.0)
+    else:
+        gate, up, down = _int4_matrix(P1, 2.0, 0.0), _int4_matrix(P2, 0.5, 0.0), _int4_matrix(P3, 1.0, 0.0)
+    rng = np.random.default_rng(1)
+    x = synth.to_bf16_bits(rng.standard_normal((M, n)))
+    res = synth.to_bf16_bits(rng.standard_normal((M, n)))
+    out = oracle.ffn_dense(FFNWeights(gate, up, down), x, res, "silu")
+    xf = oracle.bf16_to_f64(x)
+    i = np.arange(n)
+    g = 2.0 * xf[:, (i + 5) % n]
+    u = 0.5 * xf
+    a = oracle.bf16(g / (1 + np.exp(-g)) * u)
+    h = a[:, (i + 17) % n]
+    want = oracle.bf16_bits(oracle.bf16_to_f64(res) + h)
+    assert np.array_equal(out, want)
+
+
+def test_int4_min_only_closed_form():
+    """All codes 0: W[n][k] = min[n][k//32], so gate . x is min times the group sums."""
+    n, K = 8, 96
+    codes = np.zeros((n, K), np.int64)
+    w = _int4_matrix(codes, 0.25, 0.0)
+    mins = (np.arange(n * 3).reshape(n, 3) - 7) * 0.0625
+    w.min[:] = mins.astype(np.float16)
+    x = np.arange(K, dtype=np.float64) / 16.0
+    got = oracle.dequant(w) @ x
+    gsum = x.reshape(3, 32).sum(axis=1)
+    assert np.allclose(got, mins @ gsum, rtol=0, atol=1e-12)
+
+
+def test_residual_is_only_tail_on_llama():
+    """out - res is the bf16 FFN output: no norm sits between FFN and stream."""
+    c = synth.scaled_config(1, H=64, I=96)
+    inp = synth.make_inputs(c, 2, 0)
+    out = oracle.bf16_to_f64(oracle.layer(inp))
+    h = oracle.bf16(oracle.ffn_hidden(inp.ffn, oracle.bf16_to_f64(inp.x), "silu"))
+    res = oracle.bf16_to_f64(inp.residual)
+    assert np.array_equal(out, oracle.bf16(res + h))
+    # A norm on h would change its RMS; the FFN output here is far from unit RMS.
+    assert abs(np.sqrt(np.mean(h ** 2)) - 1.0) > 0.1
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 5])
+def test_zero_input_leaves_residual(cfg):
+    c = synth.scaled_config(cfg, H=64, I=64) if cfg != 5 else synth.scaled_config(5, H=64, I=64, E=4)
+    inp = synth.make_inputs(c, 2, 0)
+    inp.x = np.zeros_like(inp.x)
+    assert np.array_equal(oracle.layer(inp), inp.residual)
+
+
+def test_zero_input_shared_expert_gives_zero():
+    c = synth.scaled_config(3, H=64, I=64)
+    inp = synth.make_inputs(c, 2, 0)
+    inp.x = np.zeros_like(inp.x)
+    assert not np.any(oracle.bf16_to_f64(oracle.layer(inp)))
+
+
+def test_zero_input_qwen_moe():
+    """x = 0: logits 0, top-k = experts 0..k-1 by the tie rule, w = 1/k, seed 0."""
+    c = synth.scaled_config(4, H=64, I=32, E=16, k=8, I_s=32)
+    inp = synth.make_inputs(c, 3, 0)
+    inp.x = np.zeros_like(inp.x)
+    out, it = oracle.moe_layer(inp, return_internals=True)
+    assert np.array_equal(it["idx"], np.tile(np.arange(8), (3, 1)))
+    assert np.all(it["w"] == 0.125)
+    assert not np.any(it["seed"])
+    assert np.array_equal(out, inp.residual)
+
+
+def test_rmsnorm_constant_row_closed_form():
+    H = 48
+    w = oracle.bf16(1.0 + np.random.default_rng(2).normal(0, 0.1, H))
+    for c in (0.5, -3.0, 1e-4):
+        h1 = np.full((1, H), oracle.bf16(np.array([c]))[0])
+        want = oracle.bf16(h1 / math.sqrt(h1[0, 0] ** 2 + 1e-6) * w)
+        assert np.array_equal(oracle.rms_norm(h1, w, 1e-6), want)
+    # Scale invariance (eps negligible): 4*h1 normalizes to the same row.
+    h1 = oracle.bf16(np.random.default_rng(3).standard_normal((1, H)))
+    assert np.allclose(oracle.rms_norm(4 * h1, w, 0.0), oracle.rms_norm(h1, w, 0.0), rtol=0, atol=0)
+
+
+def test_shared_expert_branch_ends_with_norm():
+    """The Gemma branch's output rows have RMS close to RMS(w) (up to bf16)."""
+    c = synth.scaled_config(3, H=128, I=64)
+    inp = synth.make_inputs(c, 2, 1)
+    out = oracle.bf16_to_f64(oracle.layer(inp))
+    w = oracle.bf16_to_f64(inp.norm_w)
+    x = oracle.bf16_to_f64(inp.x)
+    h1 = oracle.bf16(oracle.ffn_hidden(inp.ffn, x, "gelu_tanh"))
+    n = h1 / np.sqrt(np.mean(h1 ** 2, axis=1, keepdims=True))
+    assert np.allclose(out, n * w, rtol=1e-2, atol=1e-2)
+
+
+# --------------------------------------------------------------------------- routing
+
+
+def _is_topk(logits_row, chosen, k):
+    """Brute-force definition: chosen beats every other expert under (logit, -index)."""
+    E = len(logits_row)
+    S = set(chosen)
+    if len(S) != k:
+        return False
+    for e in S:
+        for o in range(E):
+            if o in S:
+                continue
+            if not (logits_row[e] > logits_row[o] or (logits_row[e] == logits_row[o] and e < o)):
+                return False
+    return True
+
+
+def test_topk_bruteforce_with_ties():
+    rng = np.random.default_rng(3)
+    for E in (2, 3, 5, 8):
+        for k in range(1, E + 1):
+            for _ in range(20):
+                logits = rng.integers(-2, 3, size=(1, E)).astype(np.float64)
+                idx, w = oracle.topk_softmax(logits, k)
+                sets = [s for s in itertools.combinations(range(E), k) if _is_topk(logits[0], s, k)]
+                assert len(sets) == 1                         # exactly one correct answer
+                assert set(idx[0]) == set(sets[0])
+                # ranks in (logit desc, index asc) order
+                keys = [(-logits[0, e], e) for e in idx[0]]
+                assert keys == sorted(keys)
+                assert abs(w.sum() - 1) < 3e-3
+
+
+def test_topk_softmax_closed_forms():
+    logits = np.array([[0.5, 0.5, 0.5, 0.5, -1.0]])
+    idx, w = oracle.topk_softmax(logits, 4)
+    assert list(idx[0]) == [0, 1, 2, 3] and np.all(w == 0.25)
+    d = 0.75
+    idx, w = oracle.topk_softmax(np.array([[0.0, d, -5.0]]), 2)
+    assert list(idx[0]) == [1, 0]
+    assert w[0, 0] == np.float16(1 / (1 + math.exp(-d)))
+    assert w[0, 1] == np.float16(math.exp(-d) / (1 + math.exp(-d)))
+
+
+def test_router_logits_one_hot_rows():
+    H, E = 32, 4
+    Wr = np.zeros((E, H), np.float32)
+    for e in range(E):
+        Wr[e, 3 * e + 1] = 2.0
+    x = synth.to_bf16_bits(np.random.default_rng(4).standard_normal((2, H)))
+    got = oracle.router_logits(Wr, x)
+    xf = oracle.bf16_to_f64(x)
+    assert np.array_equal(got, 2.0 * xf[:, [1, 4, 7, 10]])
+
+
+def test_permutation_invariants():
+    rng = np.random.default_rng(7)
+    for M, k, E in [(1, 8, 128), (4, 8, 128), (37, 2, 8), (512, 2, 8), (5, 3, 4)]:
+        idx = np.stack([rng.choice(E, k, replace=False) for _ in range(M)]).astype(np.int32)
+        perm, offsets, union = oracle.expert_permutation(idx, E)
+        flat = idx.reshape(-1)
+        assert sorted(perm.tolist()) == list(range(M * k))                 # a permutation
+        ex = flat[perm]
+        assert np.all(np.diff(ex) >= 0)                                    # grouped by expert
+        for e in range(E):
+            seg = perm[offsets[e]:offsets[e + 1]]
+            assert np.all(np.diff(seg) > 0)                                # stable in pair order
+            assert np.all(flat[seg] == e)
+            assert len(seg) == int(np.sum(flat == e))
+        assert offsets[0] == 0 and offsets[-1] == M * k
+        assert list(union) == sorted(set(flat.tolist()))
+
+
+# --------------------------------------------------------------------------- seeded sum
+
+
+def _seed_counterexample_inputs():
+    """Hand-built layer where the seed order decides the result (exact in fp32).
+
+    H = I = 32, E = 2, k = 2, zero router (equal logits: experts 0, 1 with
+    weights 1/2, 1/2), x = e_0, shared output 2 at row 0 with w_sg = 0
+    (sigmoid = 1/2, seed = 1), expert 0 gives d = 2^-23 and expert 1 gives -2
+    at row 0, residual 0.
+    """
+    H = I = 32
+    c = synth.scaled_config(4, H=H, I=I, E=2, k=2, I_s=I)
+    z = lambda N, K: synth.zero_like_qweight(FMT_INT4_G32, N, K)   # noqa: E731
+
+    def ffn(gate00, up00, down00):
+        g, u, d = z(I, H), z(I, H), z(H, I)
+        for w, (q, s, m) in ((g, gate00), (u, up00), (d, down00)):
+            w.q[0, 0] = q
+            w.scale[0, 0] = s
+            w.min[0, 0] = m
+        return FFNWeights(g, u, d)
+
+    # gate row 0 = 64 (15*4+4) -> silu(64) = 64; up row 0 = 2^-6 -> a_0 = 1.
+    gate, up = (15, 4.0, 4.0), (1, 2.0 ** -6, 0.0)
+    shared = ffn(gate, up, (1, 2.0, 0.0))                  # s_0 = 2
+    e0 = ffn(gate, up, (2, 2.0 ** -24, 0.0))              # d_0 = 2^-23
+    e1 = ffn(gate, up, (0, 0.0, -2.0))                    # d_1 = -2
+    # min of other entries in group 0 of the gate row is 4, but x is zero there.
+    x = np.zeros((1, H), np.uint16)
+    x[0, 0] = 0x3F80
+    li = synth.LayerInputs(c, 1, 0, x, np.zeros((1, H), np.uint16), router=np.zeros((2, H), np.float32),
+                           experts=[e0, e1], shared=shared, w_sg=np.zeros(H, np.uint16))
+    return li
+
+
+def test_seed_is_accumulator_start_not_addend():
+    li = _seed_counterexample_inputs()
+    out, it = oracle.moe_layer(li, return_internals=True)
+    assert list(it["idx"][0]) == [0, 1] and np.all(it["w"] == 0.5)
+    assert it["seed"][0, 0] == 1.0
+    assert it["d"][0, 0, 0] == 2.0 ** -23 and it["d"][0, 1, 0] == -2.0
+    assert oracle.bf16_to_f64(out)[0, 0] == 0.0                      # seed, then ranks
+    # Adding the shared expert after the routed sum gives another function.
+    routed = np.float32(np.float32(0.5) * np.float32(2.0 ** -23)) + np.float32(np.float32(0.5) * np.float32(-2.0))
+    add_after = np.float32(routed + np.float32(1.0))
+    assert add_after == np.float32(2.0 ** -24)
+
+
+def test_moe_single_expert_reduces_to_dense():
+    """E = 1, k = 1, no shared expert: the routed layer is the dense FFN (w = 1)."""
+    c = synth.scaled_config(5, H=64, I=96, E=1, k=1)
+    inp = synth.make_inputs(c, 3, 2)
+    moe = oracle.bf16_to_f64(oracle.layer(inp))
+    dense = oracle.bf16_to_f64(oracle.ffn_dense(inp.experts[0], inp.x, inp.residual, "silu"))
+    # identical up to the fp32 rounding of d before the bf16 rounding of y
+    assert np.max(np.abs(moe - dense) / np.maximum(np.abs(dense), 1e-3)) <= 2.0 ** -7
+
+
+def test_moe_token_rows_independent():
+    """Rows are independent: M-row output equals the single-row outputs."""
+    c = synth.scaled_config(4, H=64, I=32, E=16, k=4, I_s=32)
+    inp = synth.make_inputs(c, 4, 1)
+    full = oracle.layer(inp)
+    for t in range(4):
+        assert np.array_equal(oracle.layer(inp, tokens=[t])[0], full[t])
