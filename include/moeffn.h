@@ -1,0 +1,203 @@
+/*
+ * moeffn.h -- C ABI of the quantized gated FFN / Mixture-of-Experts layer
+ * library for NVIDIA B200 (sm_100a), libmoeffn.so.
+ *
+ * The layer computed is the FFN half of a transformer layer as three model
+ * families run it in the turbospark-runtime pages:
+ *
+ *   h = down_proj( act(gate_proj @ m) * (up_proj @ m) )
+ *     llama / Mistral dense layer: x = x + h (raw residual add only)
+ *       -- turbospark-runtime 0.3.0, src/families/llama/dense.rs, module doc
+ *          formula box and encode_llama_layer_dense;
+ *     Gemma shared-expert branch: h1 = RMSNorm(h) * w, eps 1e-6
+ *       -- turbospark-runtime 0.1.0, src/families/gemma4/shared_expert.rs,
+ *          encode_shared_expert_branch[_batched];
+ *     Qwen-style routed MoE: top-k experts per token, phase-2 accumulator
+ *       seeded with the sigmoid-gated shared expert, ranks added in pair order,
+ *       then one raw residual add
+ *       -- turbospark-runtime 0.3.0, src/families/qwen/moe_batch.rs, module doc
+ *          and encode_qwen_layer_moe_batched.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees them and keeps none after the call returns (plans excepted:
+ *    a plan keeps the expert weight pointers until moe_plan_destroy).
+ *  - Activations are bf16 (uint16 bit patterns), token-major [M][H], rows
+ *    contiguous. x must not alias the output (the pages: the normed input
+ *    "must not be the destination of anything encoded in between").
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and never synchronize the host. No call reads results
+ *    back to the host (the reference's blocking router readback is not
+ *    reproduced).
+ *  - Hot calls allocate no memory: scratch comes from the caller's workspace
+ *    (`ws`, `ws_bytes`, 256-byte aligned, size from the *_workspace_bytes
+ *    queries). Its contents need no initialisation and are garbage after.
+ *  - Arguments are validated on the host before any launch. Unsupported
+ *    combinations are refused with MOEFFN_ERR_UNSUPPORTED and a message; there
+ *    is no fallback path (the pages' "refuse rather than degrade").
+ *  - On error the return value is negative and moeffn_last_error() gives a
+ *    thread-local message. CUDA launch errors map to MOEFFN_ERR_CUDA.
+ *
+ * Weight formats (struct moeffn_qweight, W[rows][cols], y = W x):
+ *  - MOEFFN_Q_INT8_ROW: q = int8 [rows][cols]; scale = fp16 [rows]; min = NULL.
+ *    W[n][k] = q[n][k] * scale[n]. cols % 16 == 0.
+ *  - MOEFFN_Q_INT4_AFFINE_G32: q = uint8 [rows][cols/2], element 2j in the low
+ *    nibble of byte j, 2j+1 in the high nibble; scale, min = fp16
+ *    [rows][cols/32]. W[n][k] = q * scale[n][k/32] + min[n][k/32]. cols % 32 == 0.
+ *  - MOEFFN_BF16 / MOEFFN_F32: plain [rows][cols] in q (router, gate vector).
+ *  All base pointers 16-byte aligned.
+ */
+#ifndef MOEFFN_H
+#define MOEFFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* moeffn_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  MOEFFN_OK = 0,
+  MOEFFN_ERR_INVALID = -1,     /* null pointer, bad shape, misalignment */
+  MOEFFN_ERR_UNSUPPORTED = -2, /* valid but not built (format, size limit) */
+  MOEFFN_ERR_WORKSPACE = -3,   /* workspace missing or too small */
+  MOEFFN_ERR_CUDA = -4         /* CUDA error (message has its string) */
+} moeffn_status;
+
+typedef enum {
+  MOEFFN_Q_INT8_ROW = 1,
+  MOEFFN_Q_INT4_AFFINE_G32 = 2,
+  MOEFFN_BF16 = 3,
+  MOEFFN_F32 = 4
+} moeffn_qformat;
+
+typedef enum { MOEFFN_ACT_SILU = 0, MOEFFN_ACT_GELU_TANH = 1 } moeffn_act;
+
+typedef enum {
+  MOEFFN_KIND_DENSE = 1,   /* ffn_dense */
+  MOEFFN_KIND_SHARED = 2,  /* ffn_shared_expert */
+  MOEFFN_KIND_ROUTER = 3,  /* moe_router_topk */
+  MOEFFN_KIND_MOE = 4      /* moe_layer (prefer moe_workspace_bytes) */
+} moeffn_kind;
+
+typedef struct moeffn_qweight {
+  int32_t format;     /* moeffn_qformat */
+  int32_t rows;       /* N: output features */
+  int32_t cols;       /* K: reduction length */
+  const void* q;      /* codes or plain values, see the format list above */
+  const void* scale;  /* fp16, NULL for BF16/F32 */
+  const void* min;    /* fp16, INT4 only, else NULL */
+} moeffn_qweight;
+
+/* One gated FFN: gate, up [I][H]; down [H][I]; all of one quantized format. */
+typedef struct moeffn_ffn {
+  moeffn_qweight gate, up, down;
+} moeffn_ffn;
+
+/* Workspace bytes for a call of `kind` with M token rows, hidden size H,
+ * intermediate width I, E experts and top_k ranks (E, top_k ignored for the
+ * dense kinds). For MOEFFN_KIND_MOE pass I = max(expert width, shared width).
+ * Returns 0 for invalid arguments. */
+size_t moeffn_workspace_bytes(int kind, int M, int H, int I, int E, int top_k);
+
+/* Thread-local text of the last error (empty string if none). */
+const char* moeffn_last_error(void);
+
+/* Dense llama-style FFN plus raw residual add, in place:
+ *   residual[t] = bf16(residual[t] + bf16(down(bf16(act(gate x_t) * (up x_t)))))
+ * turbospark-runtime 0.3.0, src/families/llama/dense.rs,
+ * encode_llama_layer_dense (gate and up GEMVs on the normed input, gated
+ * activation, down GEMV into h2, residual add into x).
+ * w: gate/up rows = I, cols = H; down rows = H, cols = I; INT8 or INT4 formats.
+ * x, residual: [M][H] bf16. act: moeffn_act. M >= 1. */
+int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act,
+              void* ws, size_t ws_bytes, moeffn_stream_t stream);
+
+/* Gemma shared-expert branch with its trailing post-FFN RMSNorm:
+ *   h1[t] = bf16(h / sqrt(mean(h^2) + eps) * norm_w), h = bf16(FFN(x_t))
+ * turbospark-runtime 0.1.0, src/families/gemma4/shared_expert.rs,
+ * encode_shared_expert_branch and encode_shared_expert_branch_batched
+ * (RMS_EPS = 1e-6, weight post_feedforward_layernorm_1).
+ * norm_w: [H] bf16. h1_out: [M][H] bf16 (written, not read). */
+int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* norm_w, float eps,
+                      uint16_t* h1_out, int M, int act, void* ws, size_t ws_bytes,
+                      moeffn_stream_t stream);
+
+/* Router GEMV, top-k softmax and (optionally) the expert-grouped pair order.
+ * logits[t][e] = router[e] . x[t] (fp32). Ranks r = 0..top_k-1 ordered by
+ * (logit desc, expert asc); topk_w[t][r] = fp16(softmax over the k selected
+ * logits), stored as float. perm lists pair indices p = t*top_k + r grouped by
+ * expert, stable in p; expert_offsets[e]..[e+1] is expert e's range of perm.
+ * turbospark-runtime 0.3.0, src/families/qwen/moe_batch.rs: router logits
+ * readback, router_topk_gemma4 with per_expert_ones, routes in PAIR order.
+ * router: MOEFFN_F32 or MOEFFN_BF16, rows = E (<= 1024), cols = H (% 8 == 0).
+ * logits_out [M][E], perm [M*top_k], expert_offsets [E+1] may be NULL
+ * (expert_offsets is required when perm is given). top_k in 1..16, <= E. */
+int moe_router_topk(const moeffn_qweight* router, const uint16_t* x, int M, int top_k,
+                    float* logits_out, int32_t* topk_idx, float* topk_w, int32_t* perm,
+                    int32_t* expert_offsets, void* ws, size_t ws_bytes, moeffn_stream_t stream);
+
+/* Description of a routed MoE layer (host memory; read by moe_plan_create). */
+typedef struct moeffn_moe_desc {
+  int32_t num_experts;                /* E */
+  int32_t top_k;                      /* k */
+  int32_t act;                        /* moeffn_act */
+  moeffn_qweight router;              /* F32 or BF16 [E][H] */
+  const moeffn_ffn* experts;          /* host array [E]; INT4-affine only */
+  const moeffn_ffn* shared;           /* NULL: no shared expert (routed sum starts at 0) */
+  const moeffn_qweight* shared_gate;  /* BF16 [1][H]; required with `shared` */
+} moeffn_moe_desc;
+
+typedef struct moeffn_moe_plan moeffn_moe_plan;
+
+/* Validates the description and copies the expert pointer tables to the
+ * device (the only library-owned memory). Blocking; not for the hot path. */
+int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan);
+int moe_plan_destroy(moeffn_moe_plan* plan);
+size_t moe_workspace_bytes(const moeffn_moe_plan* plan, int M);
+
+/* Routed MoE layer plus its single raw residual add, in place:
+ *   y[t] = bf16( ((seed[t] + w_0 d_0) + w_1 d_1) + ... )  (fp32, rank order)
+ *   residual[t] = bf16(residual[t] + y[t])
+ * seed = bf16(bf16(shared(x_t)) * sigmoid(shared_gate . x_t)), or 0.
+ * turbospark-runtime 0.3.0, src/families/qwen/moe_batch.rs, module doc ("this
+ * family's phase 2 SEEDS its accumulator with the gated shared-expert output",
+ * "NO SANDWICH NORMS") and encode_qwen_layer_moe_batched.
+ * topk_idx_out: optional [M][k] int32 copy of the selected experts. */
+int moe_layer(moeffn_moe_plan* plan, const uint16_t* x, uint16_t* residual, int M, int32_t* topk_idx_out,
+              void* ws, size_t ws_bytes, moeffn_stream_t stream);
+
+/* ---- Per-launch timing (tracing) ------------------------------------------
+ * No counterpart on the pages (they time host phases with PhaseCounters).
+ * Off by default. While enabled, every kernel launch of the library is
+ * bracketed by two CUDA events on its stream (a small gap per launch).
+ * moeffn_profile_read waits for the recorded events and returns, per kernel
+ * name (names: '\n'-separated, truncated to names_len), the number of
+ * launches and their summed device time in ms since the previous read, then
+ * clears the records. Not thread-safe across concurrent callers' reads. */
+int moeffn_profile_enable(int on);
+int moeffn_profile_read(char* names, int names_len, int32_t* counts, float* total_ms, int max_kernels,
+                        int* n_kernels);
+
+/* ---- Test exports: feed identical inputs to single steps. ---------------- */
+
+/* Dequantize W on the device with the kernels' own conversion: out_f32
+ * [rows][cols] (exact q*scale(+min)) and/or out_bf16 [rows][cols] (round to
+ * nearest even of the fp32 value). Either output may be NULL. */
+int moeffn_test_dequant(const moeffn_qweight* w, float* out_f32, uint16_t* out_bf16, moeffn_stream_t stream);
+
+/* Top-k, softmax weights and grouped permutation from given fp32 logits
+ * [M][E] (device). union_out [E] and n_union_out [1] may be NULL. */
+int moeffn_test_topk_from_logits(const float* logits, int M, int E, int top_k, int32_t* topk_idx,
+                                 float* topk_w, int32_t* perm, int32_t* expert_offsets,
+                                 int32_t* union_out, int32_t* n_union_out, moeffn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEFFN_H */

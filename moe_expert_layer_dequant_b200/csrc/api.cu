@@ -1,0 +1,657 @@
+// C ABI of libmoeffn.so: argument validation, workspace carving and the
+// launch sequence of each layer kind. See include/moeffn.h for the contract.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+#include <vector>
+
+#include "../../include/moeffn.h"
+#include "common.cuh"
+#include "gemv.cuh"
+#include "prof.cuh"
+#include "route.cuh"
+#include "tail.cuh"
+
+using namespace moeffn;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(MOEFFN_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define MOEFFN_CHECK_CUDA(expr, where)              \
+  do {                                              \
+    cudaError_t e_ = (expr);                        \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+constexpr int kSMs = 148;
+constexpr size_t kAlign = 256;
+constexpr size_t kStageBudget = 96 * 1024;      // shared memory per CTA for staged tokens
+constexpr size_t kStageMax = 200 * 1024;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+QW to_qw(const moeffn_qweight& w) {
+  return QW{static_cast<const uint8_t*>(w.q), static_cast<const __half*>(w.scale),
+            static_cast<const __half*>(w.min)};
+}
+
+int check_qweight(const moeffn_qweight& w, const char* name, int rows, int cols) {
+  if (w.format != MOEFFN_Q_INT8_ROW && w.format != MOEFFN_Q_INT4_AFFINE_G32)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: format %d is not INT8_ROW or INT4_AFFINE_G32", name, w.format);
+  if (w.rows != rows || w.cols != cols)
+    return fail(MOEFFN_ERR_INVALID, "%s: shape [%d][%d], expected [%d][%d]", name, w.rows, w.cols, rows, cols);
+  if (w.q == nullptr || w.scale == nullptr)
+    return fail(MOEFFN_ERR_INVALID, "%s: null q or scale", name);
+  if (!aligned16(w.q)) return fail(MOEFFN_ERR_INVALID, "%s: q is not 16-byte aligned", name);
+  if ((reinterpret_cast<uintptr_t>(w.scale) & 1u) != 0) return fail(MOEFFN_ERR_INVALID, "%s: scale misaligned", name);
+  if (w.format == MOEFFN_Q_INT4_AFFINE_G32) {
+    if (cols % 32 != 0) return fail(MOEFFN_ERR_INVALID, "%s: INT4-affine needs cols %% 32 == 0 (cols=%d)", name, cols);
+    if (w.min == nullptr) return fail(MOEFFN_ERR_INVALID, "%s: INT4-affine needs a min array", name);
+    if ((reinterpret_cast<uintptr_t>(w.min) & 1u) != 0) return fail(MOEFFN_ERR_INVALID, "%s: min misaligned", name);
+  } else if (cols % 16 != 0) {
+    return fail(MOEFFN_ERR_INVALID, "%s: INT8 needs cols %% 16 == 0 (cols=%d)", name, cols);
+  }
+  return MOEFFN_OK;
+}
+
+int check_ffn(const moeffn_ffn& f, const char* name, int H, int I) {
+  std::string n = name;
+  int rc;
+  if ((rc = check_qweight(f.gate, (n + ".gate").c_str(), I, H)) != MOEFFN_OK) return rc;
+  if ((rc = check_qweight(f.up, (n + ".up").c_str(), I, H)) != MOEFFN_OK) return rc;
+  if ((rc = check_qweight(f.down, (n + ".down").c_str(), H, I)) != MOEFFN_OK) return rc;
+  if (f.gate.format != f.up.format || f.gate.format != f.down.format)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: gate/up/down formats differ", name);
+  return MOEFFN_OK;
+}
+
+// ---- launch geometry -------------------------------------------------------
+
+int round_up8(int v) { return (v + 7) / 8 * 8; }
+
+// Rows per CTA so that about two CTAs per SM are launched.
+int rows_per_cta(int rows_total) {
+  int r = round_up8((rows_total + 2 * kSMs - 1) / (2 * kSMs));
+  return std::min(64, std::max(8, r));
+}
+
+// K split of a down projection: slices of at most about 2048 elements, a
+// multiple of 32; every split starts below K.
+int down_slice(int K) {
+  const int s = (K + 2047) / 2048;
+  return ((K + s - 1) / s + 31) / 32 * 32;
+}
+int down_splits(int K) {
+  const int ks = down_slice(K);
+  return (K + ks - 1) / ks;
+}
+
+int stage_tokens(int fmt, int klen, int want) {
+  const size_t per = gemv_stage_bytes(fmt, klen, 1);
+  int t = (int)std::max<size_t>(1, kStageBudget / per);
+  return std::max(1, std::min(want, t));
+}
+
+int mt_for(int tokens) { return tokens <= 1 ? 1 : 2; }
+
+// ---- workspace layout ------------------------------------------------------
+
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t count) {
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off = align_up(off + count * sizeof(T));
+    return p;
+  }
+};
+
+struct DenseWS {
+  uint16_t* acts;
+  float* d;
+};
+
+DenseWS carve_dense(Carve& c, int M, int H, int I) {
+  DenseWS w;
+  w.acts = c.take<uint16_t>((size_t)M * I);
+  w.d = c.take<float>((size_t)down_splits(I) * M * H);
+  return w;
+}
+
+struct MoeWS {
+  float* logits;
+  float* gate_logit;
+  int* idx;
+  float* w;
+  int* perm;
+  int* inv;
+  int* offsets;
+  int* union_list;
+  int* n_union;
+  uint16_t* acts;
+  uint16_t* acts_s;
+  float* d;
+  float* d_s;
+};
+
+// Down-projection K split shared by the routed and the shared expert jobs.
+struct MoeSplit {
+  int ks_len, routed, shared;
+};
+
+MoeSplit moe_split(int Ie, int Is) {
+  MoeSplit s;
+  s.ks_len = down_slice(std::max(Ie, Is));
+  s.routed = (Ie + s.ks_len - 1) / s.ks_len;
+  s.shared = Is > 0 ? (Is + s.ks_len - 1) / s.ks_len : 0;
+  return s;
+}
+
+MoeWS carve_moe(Carve& c, int M, int H, int Ie, int Is, int E, int k) {
+  MoeWS w;
+  const MoeSplit sp = moe_split(Ie, Is);
+  const size_t P = (size_t)M * k;
+  w.logits = c.take<float>((size_t)M * E);
+  w.gate_logit = c.take<float>(M);
+  w.idx = c.take<int>(P);
+  w.w = c.take<float>(P);
+  w.perm = c.take<int>(P);
+  w.inv = c.take<int>(P);
+  w.offsets = c.take<int>(E + 1);
+  w.union_list = c.take<int>(E);
+  w.n_union = c.take<int>(1);
+  w.acts = c.take<uint16_t>(P * Ie);
+  w.acts_s = c.take<uint16_t>((size_t)M * std::max(Is, 0));
+  w.d = c.take<float>((size_t)sp.routed * P * H);
+  w.d_s = c.take<float>((size_t)sp.shared * M * H);
+  return w;
+}
+
+struct RouterWS {
+  float* logits;
+  int* perm;
+  int* offsets;
+};
+
+RouterWS carve_router(Carve& c, int M, int E, int k) {
+  RouterWS w;
+  w.logits = c.take<float>((size_t)M * E);
+  w.perm = c.take<int>((size_t)M * k);
+  w.offsets = c.take<int>(E + 1);
+  return w;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return MOEFFN_OK;
+  if (ws == nullptr) return fail(MOEFFN_ERR_WORKSPACE, "workspace is null (%zu bytes needed)", need);
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign != 0) return fail(MOEFFN_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  if (ws_bytes < need) return fail(MOEFFN_ERR_WORKSPACE, "workspace %zu bytes, %zu needed", ws_bytes, need);
+  return MOEFFN_OK;
+}
+
+// ---- shared FFN launch (dense mode) ---------------------------------------
+
+int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, int act, const DenseWS& w,
+                  cudaStream_t s) {
+  const int fmt = f.gate.format;
+  GateUpArgs g{};
+  g.fmt = fmt;
+  g.act = act;
+  g.K = H;
+  g.g = to_qw(f.gate);
+  g.u = to_qw(f.up);
+  g.N = I;
+  g.x = x;
+  g.M = M;
+  g.topk = 1;
+  g.routed_jobs = 1;
+  g.out = w.acts;
+  g.rows_per_cta = rows_per_cta(I);
+  g.stage_tokens = stage_tokens(fmt, H, M);
+  {
+    ProfScope ps("gateup_gemv", s);
+    MOEFFN_CHECK_CUDA(launch_gateup(g, (I + g.rows_per_cta - 1) / g.rows_per_cta, 1, mt_for(M), s), "gate/up launch");
+  }
+
+  DownArgs d{};
+  d.fmt = fmt;
+  d.K = I;
+  d.N = H;
+  d.w = to_qw(f.down);
+  d.in = w.acts;
+  d.M = M;
+  d.slots = M;
+  d.d = w.d;
+  d.ks_len = down_slice(I);
+  const int splits = down_splits(I);
+  d.rows_per_cta = rows_per_cta(H * splits);
+  d.stage_tokens = stage_tokens(fmt, d.ks_len, M);
+  {
+    ProfScope ps("down_gemv", s);
+    MOEFFN_CHECK_CUDA(launch_down(d, (H + d.rows_per_cta - 1) / d.rows_per_cta, splits, 1, mt_for(M), s),
+                      "down launch");
+  }
+  return MOEFFN_OK;
+}
+
+}  // namespace
+
+// ============================================================================
+// Plan
+// ============================================================================
+
+struct moeffn_moe_plan {
+  int E, k, act, H, Ie, Is;
+  int router_fmt;
+  const void* router;
+  const uint16_t* w_sg;
+  moeffn_ffn shared;
+  bool has_shared;
+  QW* d_gate = nullptr;   // device tables [E]
+  QW* d_up = nullptr;
+  QW* d_down = nullptr;
+};
+
+extern "C" {
+
+const char* moeffn_last_error(void) { return g_last_error.c_str(); }
+
+size_t moeffn_workspace_bytes(int kind, int M, int H, int I, int E, int top_k) {
+  if (M < 1 || H < 1) return 0;
+  Carve c{nullptr};
+  switch (kind) {
+    case MOEFFN_KIND_DENSE:
+    case MOEFFN_KIND_SHARED:
+      if (I < 1) return 0;
+      carve_dense(c, M, H, I);
+      return c.off;
+    case MOEFFN_KIND_ROUTER:
+      if (E < 1 || top_k < 1) return 0;
+      carve_router(c, M, E, top_k);
+      return c.off;
+    case MOEFFN_KIND_MOE:
+      if (I < 1 || E < 1 || top_k < 1) return 0;
+      carve_moe(c, M, H, I, I, E, top_k);
+      return c.off;
+    default:
+      return 0;
+  }
+}
+
+int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act, void* ws,
+              size_t ws_bytes, moeffn_stream_t stream) {
+  g_last_error.clear();
+  if (w == nullptr || x == nullptr || residual == nullptr) return fail(MOEFFN_ERR_INVALID, "ffn_dense: null pointer");
+  if (M < 1) return fail(MOEFFN_ERR_INVALID, "ffn_dense: M=%d", M);
+  if (act != MOEFFN_ACT_SILU && act != MOEFFN_ACT_GELU_TANH) return fail(MOEFFN_ERR_INVALID, "ffn_dense: act=%d", act);
+  const int H = w->gate.cols, I = w->gate.rows;
+  int rc = check_ffn(*w, "ffn_dense", H, I);
+  if (rc != MOEFFN_OK) return rc;
+  if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "ffn_dense: x/residual not 16-byte aligned");
+  if (x == residual) return fail(MOEFFN_ERR_INVALID, "ffn_dense: x aliases residual");
+  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax || gemv_stage_bytes(w->gate.format, down_slice(I), 1) > kStageMax)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "ffn_dense: hidden size %d too large for the staged GEMV", H);
+  Carve c{nullptr};
+  carve_dense(c, M, H, I);
+  if ((rc = check_ws(ws, ws_bytes, c.off)) != MOEFFN_OK) return rc;
+  Carve cw{static_cast<char*>(ws)};
+  const DenseWS d = carve_dense(cw, M, H, I);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s)) != MOEFFN_OK) return rc;
+  TailArgs t{};
+  t.mode = TAIL_RESIDUAL;
+  t.M = M;
+  t.N = H;
+  t.d = d.d;
+  t.splits = down_splits(I);
+  t.slots = M;
+  t.res = residual;
+  {
+    ProfScope ps("tail_residual", s);
+    MOEFFN_CHECK_CUDA(launch_tail(t, s), "residual tail launch");
+  }
+  return MOEFFN_OK;
+}
+
+int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* norm_w, float eps, uint16_t* h1_out,
+                      int M, int act, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
+  g_last_error.clear();
+  if (w == nullptr || x == nullptr || norm_w == nullptr || h1_out == nullptr)
+    return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: null pointer");
+  if (M < 1) return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: M=%d", M);
+  if (act != MOEFFN_ACT_SILU && act != MOEFFN_ACT_GELU_TANH)
+    return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: act=%d", act);
+  if (!(eps >= 0.0f)) return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: eps must be >= 0");
+  const int H = w->gate.cols, I = w->gate.rows;
+  int rc = check_ffn(*w, "ffn_shared_expert", H, I);
+  if (rc != MOEFFN_OK) return rc;
+  if (!aligned16(x) || !aligned16(h1_out)) return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: x/h1 not 16-byte aligned");
+  if (x == h1_out) return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: x aliases h1_out");
+  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "ffn_shared_expert: hidden size %d too large", H);
+  Carve c{nullptr};
+  carve_dense(c, M, H, I);
+  if ((rc = check_ws(ws, ws_bytes, c.off)) != MOEFFN_OK) return rc;
+  Carve cw{static_cast<char*>(ws)};
+  const DenseWS d = carve_dense(cw, M, H, I);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s)) != MOEFFN_OK) return rc;
+  TailArgs t{};
+  t.mode = TAIL_RMSNORM;
+  t.M = M;
+  t.N = H;
+  t.d = d.d;
+  t.splits = down_splits(I);
+  t.slots = M;
+  t.h1 = h1_out;
+  t.norm_w = norm_w;
+  t.eps = eps;
+  {
+    ProfScope ps("tail_rmsnorm", s);
+    MOEFFN_CHECK_CUDA(launch_tail(t, s), "rmsnorm tail launch");
+  }
+  return MOEFFN_OK;
+}
+
+static int check_router(const moeffn_qweight* router, int H_expected, const char* who) {
+  if (router == nullptr || router->q == nullptr) return fail(MOEFFN_ERR_INVALID, "%s: null router", who);
+  if (router->format != MOEFFN_F32 && router->format != MOEFFN_BF16)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: router format %d is not F32 or BF16", who, router->format);
+  if (router->rows < 1 || router->rows > kMaxExperts)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: %d experts (1..%d supported)", who, router->rows, kMaxExperts);
+  if (H_expected >= 0 && router->cols != H_expected)
+    return fail(MOEFFN_ERR_INVALID, "%s: router cols %d != hidden %d", who, router->cols, H_expected);
+  if (router->cols % 8 != 0) return fail(MOEFFN_ERR_INVALID, "%s: hidden size must be a multiple of 8", who);
+  if (!aligned16(router->q)) return fail(MOEFFN_ERR_INVALID, "%s: router not 16-byte aligned", who);
+  return MOEFFN_OK;
+}
+
+int moe_router_topk(const moeffn_qweight* router, const uint16_t* x, int M, int top_k, float* logits_out,
+                    int32_t* topk_idx, float* topk_w, int32_t* perm, int32_t* expert_offsets, void* ws,
+                    size_t ws_bytes, moeffn_stream_t stream) {
+  g_last_error.clear();
+  int rc = check_router(router, -1, "moe_router_topk");
+  if (rc != MOEFFN_OK) return rc;
+  const int E = router->rows, H = router->cols;
+  if (x == nullptr || topk_idx == nullptr || topk_w == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_router_topk: null pointer");
+  if (!aligned16(x)) return fail(MOEFFN_ERR_INVALID, "moe_router_topk: x not 16-byte aligned");
+  if (M < 1) return fail(MOEFFN_ERR_INVALID, "moe_router_topk: M=%d", M);
+  if (top_k < 1 || top_k > kMaxTopK || top_k > E)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "moe_router_topk: top_k=%d (1..%d and <= E=%d)", top_k, kMaxTopK, E);
+  if (perm != nullptr && expert_offsets == nullptr)
+    return fail(MOEFFN_ERR_INVALID, "moe_router_topk: perm needs expert_offsets");
+  Carve c{nullptr};
+  carve_router(c, M, E, top_k);
+  if ((rc = check_ws(ws, ws_bytes, c.off)) != MOEFFN_OK) return rc;
+  Carve cw{static_cast<char*>(ws)};
+  const RouterWS w = carve_router(cw, M, E, top_k);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  RouterArgs ra{};
+  ra.router = router->q;
+  ra.router_f32 = router->format == MOEFFN_F32;
+  ra.x = x;
+  ra.M = M;
+  ra.H = H;
+  ra.E = E;
+  ra.logits = logits_out != nullptr ? logits_out : w.logits;
+  {
+    ProfScope ps("router_logits", s);
+    MOEFFN_CHECK_CUDA(launch_router_logits(ra, s), "router launch");
+  }
+  RouteArgs rt{};
+  rt.logits = ra.logits;
+  rt.M = M;
+  rt.E = E;
+  rt.k = top_k;
+  rt.idx = topk_idx;
+  rt.w = topk_w;
+  rt.perm = perm;
+  rt.offsets = expert_offsets;
+  {
+    ProfScope ps("route_topk", s);
+    MOEFFN_CHECK_CUDA(launch_route(rt, s), "top-k launch");
+  }
+  return MOEFFN_OK;
+}
+
+int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
+  g_last_error.clear();
+  if (desc == nullptr || plan == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_plan_create: null pointer");
+  *plan = nullptr;
+  int rc = check_router(&desc->router, -1, "moe_plan_create");
+  if (rc != MOEFFN_OK) return rc;
+  const int E = desc->num_experts, k = desc->top_k, H = desc->router.cols;
+  if (E != desc->router.rows) return fail(MOEFFN_ERR_INVALID, "moe_plan_create: num_experts %d != router rows %d", E, desc->router.rows);
+  if (k < 1 || k > kMaxTopK || k > E) return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: top_k=%d", k);
+  if (desc->act != MOEFFN_ACT_SILU && desc->act != MOEFFN_ACT_GELU_TANH)
+    return fail(MOEFFN_ERR_INVALID, "moe_plan_create: act=%d", desc->act);
+  if (desc->experts == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_plan_create: null experts");
+  const int Ie = desc->experts[0].gate.rows;
+  std::vector<QW> g(E), u(E), d(E);
+  for (int e = 0; e < E; ++e) {
+    char name[64];
+    snprintf(name, sizeof(name), "expert[%d]", e);
+    if ((rc = check_ffn(desc->experts[e], name, H, Ie)) != MOEFFN_OK) return rc;
+    if (desc->experts[e].gate.format != MOEFFN_Q_INT4_AFFINE_G32)
+      return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: %s is not INT4-affine (the routed path takes INT4-affine blobs only)", name);
+    g[e] = to_qw(desc->experts[e].gate);
+    u[e] = to_qw(desc->experts[e].up);
+    d[e] = to_qw(desc->experts[e].down);
+  }
+  int Is = 0;
+  if (desc->shared != nullptr) {
+    Is = desc->shared->gate.rows;
+    if ((rc = check_ffn(*desc->shared, "shared", H, Is)) != MOEFFN_OK) return rc;
+    if (desc->shared->gate.format != MOEFFN_Q_INT4_AFFINE_G32 && desc->shared->gate.format != MOEFFN_Q_INT8_ROW)
+      return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: shared format");
+    if (desc->shared_gate == nullptr || desc->shared_gate->q == nullptr || desc->shared_gate->format != MOEFFN_BF16 ||
+        desc->shared_gate->cols != H || desc->shared_gate->rows != 1 || !aligned16(desc->shared_gate->q))
+      return fail(MOEFFN_ERR_INVALID, "moe_plan_create: shared expert needs a BF16 [1][H] 16-byte aligned shared_gate");
+  } else if (desc->shared_gate != nullptr) {
+    return fail(MOEFFN_ERR_INVALID, "moe_plan_create: shared_gate without a shared expert");
+  }
+  if (gemv_stage_bytes(MOEFFN_Q_INT4_AFFINE_G32, H, 1) > kStageMax)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: hidden size %d too large", H);
+  auto* p = new moeffn_moe_plan();
+  p->E = E; p->k = k; p->act = desc->act; p->H = H; p->Ie = Ie; p->Is = Is;
+  p->router_fmt = desc->router.format;
+  p->router = desc->router.q;
+  p->has_shared = desc->shared != nullptr;
+  if (p->has_shared) {
+    p->shared = *desc->shared;
+    p->w_sg = static_cast<const uint16_t*>(desc->shared_gate->q);
+  }
+  cudaError_t e1 = cudaMalloc(&p->d_gate, sizeof(QW) * E);
+  cudaError_t e2 = cudaMalloc(&p->d_up, sizeof(QW) * E);
+  cudaError_t e3 = cudaMalloc(&p->d_down, sizeof(QW) * E);
+  if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
+    moe_plan_destroy(p);
+    return fail(MOEFFN_ERR_CUDA, "moe_plan_create: cudaMalloc of the pointer tables failed");
+  }
+  cudaError_t e4 = cudaMemcpy(p->d_gate, g.data(), sizeof(QW) * E, cudaMemcpyHostToDevice);
+  cudaError_t e5 = cudaMemcpy(p->d_up, u.data(), sizeof(QW) * E, cudaMemcpyHostToDevice);
+  cudaError_t e6 = cudaMemcpy(p->d_down, d.data(), sizeof(QW) * E, cudaMemcpyHostToDevice);
+  if (e4 != cudaSuccess || e5 != cudaSuccess || e6 != cudaSuccess) {
+    moe_plan_destroy(p);
+    return fail(MOEFFN_ERR_CUDA, "moe_plan_create: copy of the pointer tables failed");
+  }
+  *plan = p;
+  return MOEFFN_OK;
+}
+
+int moe_plan_destroy(moeffn_moe_plan* plan) {
+  if (plan == nullptr) return MOEFFN_OK;
+  cudaFree(plan->d_gate);
+  cudaFree(plan->d_up);
+  cudaFree(plan->d_down);
+  delete plan;
+  return MOEFFN_OK;
+}
+
+size_t moe_workspace_bytes(const moeffn_moe_plan* p, int M) {
+  if (p == nullptr || M < 1) return 0;
+  Carve c{nullptr};
+  carve_moe(c, M, p->H, p->Ie, p->Is, p->E, p->k);
+  return c.off;
+}
+
+int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, int32_t* topk_idx_out, void* ws,
+              size_t ws_bytes, moeffn_stream_t stream) {
+  g_last_error.clear();
+  if (p == nullptr || x == nullptr || residual == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_layer: null pointer");
+  if (M < 1) return fail(MOEFFN_ERR_INVALID, "moe_layer: M=%d", M);
+  if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "moe_layer: x/residual not 16-byte aligned");
+  if (x == residual) return fail(MOEFFN_ERR_INVALID, "moe_layer: x aliases residual");
+  const int E = p->E, k = p->k, H = p->H, Ie = p->Ie, Is = p->Is;
+  Carve c{nullptr};
+  carve_moe(c, M, H, Ie, Is, E, k);
+  int rc = check_ws(ws, ws_bytes, c.off);
+  if (rc != MOEFFN_OK) return rc;
+  Carve cw{static_cast<char*>(ws)};
+  const MoeWS w = carve_moe(cw, M, H, Ie, Is, E, k);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int P = M * k;
+
+  RouterArgs ra{};
+  ra.router = p->router;
+  ra.router_f32 = p->router_fmt == MOEFFN_F32;
+  ra.w_sg = p->has_shared ? p->w_sg : nullptr;
+  ra.x = x;
+  ra.M = M;
+  ra.H = H;
+  ra.E = E;
+  ra.logits = w.logits;
+  ra.gate_logit = w.gate_logit;
+  {
+    ProfScope ps("router_logits", s);
+    MOEFFN_CHECK_CUDA(launch_router_logits(ra, s), "router launch");
+  }
+
+  RouteArgs rt{};
+  rt.logits = w.logits;
+  rt.M = M;
+  rt.E = E;
+  rt.k = k;
+  rt.idx = topk_idx_out != nullptr ? topk_idx_out : w.idx;
+  rt.w = w.w;
+  rt.perm = w.perm;
+  rt.inv = w.inv;
+  rt.offsets = w.offsets;
+  rt.union_list = w.union_list;
+  rt.n_union = w.n_union;
+  {
+    ProfScope ps("route_topk", s);
+    MOEFFN_CHECK_CUDA(launch_route(rt, s), "route launch");
+  }
+
+  const int routed_jobs = std::min(E, P);
+  const int jobs = routed_jobs + (p->has_shared ? 1 : 0);
+  const int max_tok = M;  // a token selects an expert at most once
+  GateUpArgs g{};
+  g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
+  g.act = p->act;
+  g.K = H;
+  g.g_tab = p->d_gate;
+  g.u_tab = p->d_up;
+  g.N = Ie;
+  if (p->has_shared) {
+    g.sg = to_qw(p->shared.gate);
+    g.su = to_qw(p->shared.up);
+    g.Ns = Is;
+  }
+  g.x = x;
+  g.M = M;
+  g.topk = k;
+  g.perm = w.perm;
+  g.offsets = w.offsets;
+  g.union_list = w.union_list;
+  g.n_union = w.n_union;
+  g.routed_jobs = routed_jobs;
+  g.out = w.acts;
+  g.out_s = w.acts_s;
+  // Expected active rows: min(E, P) experts of Ie rows (+ the shared expert).
+  g.rows_per_cta = rows_per_cta(std::min(E, P) * Ie + Is);
+  g.stage_tokens = stage_tokens(g.fmt, H, max_tok);
+  if (p->has_shared && p->shared.gate.format != MOEFFN_Q_INT4_AFFINE_G32)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "moe_layer: shared expert must share the routed format");
+  const int gx = (std::max(Ie, Is) + g.rows_per_cta - 1) / g.rows_per_cta;
+  {
+    ProfScope ps("phase1_gateup_gemv", s);
+    MOEFFN_CHECK_CUDA(launch_gateup(g, gx, jobs, mt_for(std::min(M, 2)), s), "phase-1 launch");
+  }
+
+  DownArgs d{};
+  d.fmt = MOEFFN_Q_INT4_AFFINE_G32;
+  d.K = Ie;
+  d.N = H;
+  d.tab = p->d_down;
+  if (p->has_shared) d.ws = to_qw(p->shared.down);
+  d.Ks = Is;
+  d.in = w.acts;
+  d.in_s = w.acts_s;
+  d.M = M;
+  d.slots = P;
+  d.offsets = w.offsets;
+  d.union_list = w.union_list;
+  d.n_union = w.n_union;
+  d.routed_jobs = routed_jobs;
+  d.d = w.d;
+  d.d_s = w.d_s;
+  // One slice length for routed and shared jobs; each job has its own count.
+  const MoeSplit sp = moe_split(Ie, Is);
+  d.ks_len = sp.ks_len;
+  const int splits_r = sp.routed, splits_sh = sp.shared;
+  d.rows_per_cta = rows_per_cta(H * std::max(1, std::min(E, P) / 4));
+  d.stage_tokens = stage_tokens(d.fmt, d.ks_len, max_tok);
+  {
+    ProfScope ps("phase2_down_gemv", s);
+    MOEFFN_CHECK_CUDA(launch_down(d, (H + d.rows_per_cta - 1) / d.rows_per_cta, std::max(splits_r, splits_sh), jobs,
+                                  mt_for(std::min(M, 2)), s),
+                      "phase-2 launch");
+  }
+
+  TailArgs t{};
+  t.mode = TAIL_MOE;
+  t.M = M;
+  t.N = H;
+  t.d = w.d;
+  t.splits = splits_r;
+  t.slots = P;
+  t.d_s = p->has_shared ? w.d_s : nullptr;
+  t.splits_s = splits_sh;
+  t.gate_logit = w.gate_logit;
+  t.w = w.w;
+  t.inv = w.inv;
+  t.k = k;
+  t.res = residual;
+  {
+    ProfScope ps("tail_moe", s);
+    MOEFFN_CHECK_CUDA(launch_tail(t, s), "moe tail launch");
+  }
+  return MOEFFN_OK;
+}
+
+}  // extern "C"
+
+namespace moeffn {
+// Error reporting for the other translation units of the library.
+int api_fail(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace moeffn

@@ -1,0 +1,77 @@
+"""Helpers of the GPU tests: upload seeded inputs, run the library, compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+import moe_expert_layer_dequant_b200 as lib
+
+RTOL_RMS = 2e-2   # max |err| <= 2e-2 * RMS(oracle output), bf16 outputs
+WTOL_REL = 1e-3   # routing weights, relative
+
+
+def dev_bf16(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda()
+
+
+def host_bf16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def rms(v: np.ndarray) -> float:
+    return float(np.sqrt(np.mean(np.asarray(v, np.float64) ** 2)))
+
+
+def assert_bf16_close(got_bits: np.ndarray, want_bits: np.ndarray, what: str = "", rtol: float = RTOL_RMS):
+    g = oracle.bf16_to_f64(got_bits)
+    w = oracle.bf16_to_f64(want_bits)
+    assert g.shape == w.shape, (g.shape, w.shape)
+    scale = rms(w)
+    err = float(np.max(np.abs(g - w))) if g.size else 0.0
+    assert err <= rtol * max(scale, 1e-30), f"{what}: max|err| {err:.3e} > {rtol} * RMS {scale:.3e}"
+    return err / max(scale, 1e-30)
+
+
+class DeviceLayer:
+    """A synth.LayerInputs uploaded to the GPU, callable through the C ABI."""
+
+    def __init__(self, inp):
+        self.inp = inp
+        c = self.c = inp.config
+        if c.kind in ("dense", "shared"):
+            self.ffn = lib.upload_ffn(inp.ffn)
+        if c.kind == "shared":
+            self.norm_w = dev_bf16(inp.norm_w)
+        if c.kind == "moe":
+            r = inp.router
+            rt = torch.from_numpy(r).cuda() if r.dtype == np.float32 else dev_bf16(r)
+            self.router = lib.plain_weight(rt)
+            self.experts = [lib.upload_ffn(e) for e in inp.experts]
+            self.shared = lib.upload_ffn(inp.shared) if inp.shared is not None else None
+            self.w_sg = lib.plain_weight(dev_bf16(inp.w_sg)) if inp.w_sg is not None else None
+            self.plan = lib.MoePlan(self.router, self.experts, c.k, c.act, self.shared, self.w_sg)
+
+    def run(self, x_bits: np.ndarray, res_bits: np.ndarray, topk_out: bool = False):
+        x = dev_bf16(x_bits)
+        res = dev_bf16(res_bits)
+        idx = None
+        if self.c.kind == "dense":
+            lib.ffn_dense(self.ffn, x, res, self.c.act)
+            out = res
+        elif self.c.kind == "shared":
+            out = torch.empty_like(x)
+            lib.ffn_shared_expert(self.ffn, x, self.norm_w, out, self.c.act, self.c.eps)
+        else:
+            idx = torch.empty((x.shape[0], self.c.k), dtype=torch.int32, device="cuda") if topk_out else None
+            lib.moe_layer(self.plan, x, res, idx)
+            out = res
+        torch.cuda.synchronize()
+        o = host_bf16(out)
+        if topk_out:
+            return o, idx.cpu().numpy()
+        return o
+
+    def close(self):
+        if self.c.kind == "moe":
+            self.plan.close()

@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI library: it loads, exports every declared
+entry point, sizes workspaces, and refuses bad arguments before any launch.
+No GPU is touched."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "moeffn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(\w+)\s*\([^;{]*\)\s*;", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_library_builds_and_loads():
+    import moe_expert_layer_dequant_b200 as lib
+    assert os.path.exists(lib.LIB_PATH)
+
+
+def test_every_declared_symbol_is_exported():
+    import moe_expert_layer_dequant_b200 as lib
+    names = declared_functions()
+    assert "ffn_dense" in names and "moe_layer" in names and "moe_router_topk" in names
+    assert "ffn_shared_expert" in names and len(names) >= 11
+    so = ctypes.CDLL(lib.LIB_PATH)
+    missing = [n for n in names if not hasattr(so, n)]
+    assert not missing, missing
+
+
+def test_workspace_sizes():
+    import moe_expert_layer_dequant_b200 as lib
+    d1 = lib.workspace_bytes(lib.KIND_DENSE, 1, 4096, 14336)
+    d16 = lib.workspace_bytes(lib.KIND_DENSE, 16, 4096, 14336)
+    assert 0 < d1 < d16
+    # activations [M][I] bf16 + fp32 K-split partials [S][M][H]
+    assert d16 >= 16 * 14336 * 2 + 7 * 16 * 4096 * 4
+    assert lib.workspace_bytes(lib.KIND_MOE, 4, 2048, 768, 128, 8) > 0
+    assert lib.workspace_bytes(lib.KIND_DENSE, 0, 4096, 14336) == 0
+    assert lib.workspace_bytes(99, 1, 4096, 14336) == 0
+
+
+# Pointer-free refusals: every call below must fail validation before any
+# CUDA call. They use fake addresses, so they only run where no GPU exists.
+nogpu = pytest.mark.skipif(torch.cuda.is_available(), reason="fake-pointer refusals run only without a GPU")
+
+
+def _fake_qweight(lib, fmt, rows, cols, base):
+    return lib._QWeight(fmt, rows, cols, base, base + 0x100000, base + 0x200000 if fmt == lib.Q_INT4_AFFINE_G32 else None)
+
+
+def _fake_ffn(lib, fmt, H, I):
+    return lib._FFN(_fake_qweight(lib, fmt, I, H, 0x10000000), _fake_qweight(lib, fmt, I, H, 0x20000000),
+                    _fake_qweight(lib, fmt, H, I, 0x30000000))
+
+
+@nogpu
+def test_refusals_before_launch():
+    import moe_expert_layer_dequant_b200 as lib
+    L = lib._lib
+    f = _fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256, 512)
+    x, r, ws = 0x40000000, 0x50000000, 0x60000000
+    need = lib.workspace_bytes(lib.KIND_DENSE, 2, 256, 512)
+    assert L.ffn_dense(None, x, r, 2, 0, ws, need, None) == -1
+    assert L.ffn_dense(ctypes.byref(f), x, r, 0, 0, ws, need, None) == -1          # M = 0
+    assert L.ffn_dense(ctypes.byref(f), x, r, 2, 7, ws, need, None) == -1          # bad act
+    assert L.ffn_dense(ctypes.byref(f), x, x, 2, 0, ws, need, None) == -1          # x aliases residual
+    assert L.ffn_dense(ctypes.byref(f), x + 2, r, 2, 0, ws, need, None) == -1      # misaligned x
+    assert L.ffn_dense(ctypes.byref(f), x, r, 2, 0, None, need, None) == -3        # no workspace
+    assert L.ffn_dense(ctypes.byref(f), x, r, 2, 0, ws, need - 1, None) == -3      # too small
+    assert L.ffn_dense(ctypes.byref(f), x, r, 2, 0, ws + 16, need, None) == -3     # misaligned workspace
+    assert b"workspace" in L.moeffn_last_error()
+    bad = _fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256 + 16, 512)                      # K % 32 != 0
+    assert L.ffn_dense(ctypes.byref(bad), x, r, 2, 0, ws, 1 << 30, None) == -1
+    fmt = _fake_ffn(lib, 9, 256, 512)                                                # unknown format
+    assert L.ffn_dense(ctypes.byref(fmt), x, r, 2, 0, ws, 1 << 30, None) == -2
+    mixed = _fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256, 512)
+    mixed.down = _fake_qweight(lib, lib.Q_INT8_ROW, 256, 512, 0x30000000)
+    assert L.ffn_dense(ctypes.byref(mixed), x, r, 2, 0, ws, 1 << 30, None) == -2
+    shape = _fake_ffn(lib, lib.Q_INT8_ROW, 256, 512)
+    shape.down = _fake_qweight(lib, lib.Q_INT8_ROW, 512, 256, 0x30000000)           # transposed down
+    assert L.ffn_dense(ctypes.byref(shape), x, r, 2, 0, ws, 1 << 30, None) == -1
+    assert b"shape" in L.moeffn_last_error()
+
+
+@nogpu
+def test_router_and_plan_refusals():
+    import moe_expert_layer_dequant_b200 as lib
+    L = lib._lib
+    router = lib._QWeight(lib.F32, 8, 256, 0x10000000, None, None)
+    x, ws = 0x40000000, 0x60000000
+    idx, w = 0x70000000, 0x71000000
+    assert L.moe_router_topk(ctypes.byref(router), x, 4, 0, None, idx, w, None, None, ws, 1 << 20, None) == -2
+    assert L.moe_router_topk(ctypes.byref(router), x, 4, 9, None, idx, w, None, None, ws, 1 << 20, None) == -2
+    assert L.moe_router_topk(ctypes.byref(router), x, 4, 2, None, idx, w, 0x72000000, None, ws, 1 << 20, None) == -1
+    int8_router = lib._QWeight(lib.Q_INT8_ROW, 8, 256, 0x10000000, 0x11000000, None)
+    assert L.moe_router_topk(ctypes.byref(int8_router), x, 4, 2, None, idx, w, None, None, ws, 1 << 20, None) == -2
+    # The routed path takes INT4-affine experts only (refuse, do not degrade).
+    experts = (lib._FFN * 8)(*[_fake_ffn(lib, lib.Q_INT8_ROW, 256, 512) for _ in range(8)])
+    desc = lib._MoeDesc(8, 2, 0, router, experts, None, None)
+    h = ctypes.c_void_p()
+    assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -2
+    assert b"INT4" in L.moeffn_last_error()
+    desc.top_k = 0
+    assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -2
+    assert L.moe_layer(None, x, 0x50000000, 1, None, ws, 1 << 20, None) == -1

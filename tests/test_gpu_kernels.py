@@ -1,0 +1,226 @@
+"""GPU parity of the single steps and of small layers against the CPU oracle.
+
+Shapes are small enough for the oracle to finish in seconds but span several
+CTA row tiles, several 16-byte chunks per lane, and ragged tails (row counts
+that are not a multiple of the tile, K that leaves lanes idle).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from conftest import read_golden
+from devutil import DeviceLayer, assert_bf16_close, dev_bf16, host_bf16, WTOL_REL
+from synth import FMT_INT4_G32, FMT_INT8_ROW
+
+pytestmark = pytest.mark.gpu
+
+lib = pytest.importorskip("moe_expert_layer_dequant_b200")
+
+
+def _qw_dev(w):
+    return lib.upload_qweight(w)
+
+
+# --------------------------------------------------------------------------- dequant (bit-exact)
+
+
+@pytest.mark.parametrize("fmt,N,K", [(FMT_INT4_G32, 37, 96), (FMT_INT8_ROW, 29, 48), (FMT_INT4_G32, 256, 4096)])
+def test_dequant_bit_exact(fmt, N, K):
+    w = synth.random_qweight(fmt, N, K, np.random.default_rng(11))
+    f32, b16 = lib.test_dequant(_qw_dev(w))
+    torch.cuda.synchronize()
+    ref = oracle.dequant(w)
+    assert np.array_equal(f32.cpu().numpy().astype(np.float64), ref)
+    assert np.array_equal(b16.cpu().numpy().view(np.uint16), oracle.bf16_bits(ref))
+
+
+def test_dequant_golden_blocks():
+    kv, _ = read_golden("int4_affine_g32_block.txt")
+    packed = np.array([int(t, 16) for t in kv["packed_hex"]], np.uint8)[None, :]
+    sc = np.array([int(t, 16) for t in kv["scale_fp16_hex"]], np.uint16).view(np.float16)[None, :]
+    mn = np.array([int(t, 16) for t in kv["min_fp16_hex"]], np.uint16).view(np.float16)[None, :]
+    w = synth.QWeight(FMT_INT4_G32, 1, 64, packed, sc, mn)
+    f32, _ = lib.test_dequant(_qw_dev(w))
+    assert np.array_equal(f32.cpu().numpy()[0].astype(np.float64), [float(t) for t in kv["expected"]])
+    kv, _ = read_golden("int8_row_block.txt")
+    q = np.array([[int(t) for t in kv["q_row0"]], [int(t) for t in kv["q_row1"]]] * 1, np.int8)
+    q = np.concatenate([q, np.zeros((2, 8), np.int8)], axis=1)  # K = 16
+    sc = np.array([int(t, 16) for t in kv["scale_fp16_hex"]], np.uint16).view(np.float16)
+    f32, _ = lib.test_dequant(_qw_dev(synth.QWeight(FMT_INT8_ROW, 2, 16, q, sc)))
+    got = f32.cpu().numpy()[:, :8].astype(np.float64)
+    assert np.array_equal(got[0], [float(t) for t in kv["expected_row0"]])
+    assert np.array_equal(got[1], [float(t) for t in kv["expected_row1"]])
+
+
+# --------------------------------------------------------------------------- top-k / permutation (bit-exact)
+
+
+@pytest.mark.parametrize("M,E,k", [(1, 128, 8), (4, 128, 8), (37, 8, 2), (512, 8, 2), (5, 3, 3), (9, 64, 1)])
+def test_topk_permutation_from_oracle_logits(M, E, k):
+    rng = np.random.default_rng(M * 1000 + E)
+    logits = oracle.f32(rng.normal(0, 1, (M, E)))
+    logits[:, ::3] = np.round(logits[:, ::3])          # force ties
+    idx, w, perm, offs, uni = lib.test_topk_from_logits(torch.from_numpy(logits.astype(np.float32)).cuda(), k)
+    torch.cuda.synchronize()
+    ridx, rw = oracle.topk_softmax(logits, k)
+    rperm, roffs, runi = oracle.expert_permutation(ridx, E)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.array_equal(perm.cpu().numpy(), rperm)
+    assert np.array_equal(offs.cpu().numpy(), roffs)
+    assert np.array_equal(uni.cpu().numpy(), runi)
+    assert np.max(np.abs(w.cpu().numpy() - rw) / rw) <= WTOL_REL
+
+
+def test_topk_all_ties_lower_index_wins():
+    logits = torch.zeros((3, 16), dtype=torch.float32, device="cuda")
+    idx, w, perm, offs, uni = lib.test_topk_from_logits(logits, 4)
+    assert np.array_equal(idx.cpu().numpy(), np.tile(np.arange(4), (3, 1)))
+    assert np.all(w.cpu().numpy() == 0.25)
+    assert np.array_equal(perm.cpu().numpy(), [0, 4, 8, 1, 5, 9, 2, 6, 10, 3, 7, 11])
+
+
+def test_router_logits_and_topk_end_to_end():
+    c = synth.scaled_config(4, H=256, I=64, E=32, k=4, I_s=64)
+    inp = synth.make_inputs(c, 6, 3)
+    router = lib.plain_weight(torch.from_numpy(inp.router).cuda())
+    logits = torch.empty((6, 32), dtype=torch.float32, device="cuda")
+    perm = torch.empty(24, dtype=torch.int32, device="cuda")
+    offs = torch.empty(33, dtype=torch.int32, device="cuda")
+    idx, w = lib.moe_router_topk(router, dev_bf16(inp.x), 4, logits, perm, offs)
+    torch.cuda.synchronize()
+    rl = oracle.router_logits(inp.router, inp.x)
+    assert np.max(np.abs(logits.cpu().numpy() - rl)) <= 1e-5 * max(1.0, np.abs(rl).max())
+    ridx, rw = oracle.topk_softmax(rl, 4)
+    srt = np.sort(rl, axis=1)[:, ::-1]
+    margin = srt[:, 3] - srt[:, 4]
+    ok = margin > 1e-4 * np.sqrt(np.mean(rl ** 2))
+    assert np.array_equal(idx.cpu().numpy()[ok], ridx[ok])
+
+
+# --------------------------------------------------------------------------- layers, small shapes
+
+
+DENSE_SMALL = [
+    (1, dict(H=256, I=416), FMT_INT8_ROW),
+    (2, dict(H=640, I=1056), FMT_INT4_G32),
+]
+
+
+@pytest.mark.parametrize("cfg,shape,fmt", DENSE_SMALL)
+@pytest.mark.parametrize("M", [1, 2, 3, 5])
+def test_dense_small(cfg, shape, fmt, M):
+    c = synth.scaled_config(cfg, **shape)
+    inp = synth.make_inputs(c, M, 0)
+    dl = DeviceLayer(inp)
+    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "out")
+    zero = np.zeros_like(inp.residual)             # residual 0: out is bf16(h), checked strictly
+    inp.residual = zero
+    assert_bf16_close(dl.run(inp.x, zero), oracle.layer(inp), "h")
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 8])
+def test_shared_expert_small(M):
+    c = synth.scaled_config(3, H=384, I=800)
+    inp = synth.make_inputs(c, M, 1)
+    dl = DeviceLayer(inp)
+    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "h1")
+
+
+MOE_SMALL = [
+    dict(cfg=4, H=256, I=96, E=16, k=4, I_s=64),
+    dict(cfg=5, H=320, I=192, E=8, k=2, I_s=0),
+    dict(cfg=4, H=256, I=64, E=4, k=4, I_s=128),
+]
+
+
+@pytest.mark.parametrize("shape", MOE_SMALL)
+@pytest.mark.parametrize("M", [1, 2, 3, 7])
+def test_moe_small(shape, M):
+    shape = dict(shape)
+    c = synth.scaled_config(shape.pop("cfg"), **shape)
+    inp = synth.make_inputs(c, M, 2)
+    dl = DeviceLayer(inp)
+    out, idx = dl.run(inp.x, inp.residual, topk_out=True)
+    ref, it = oracle.moe_layer(inp, return_internals=True)
+    assert np.array_equal(idx, it["idx"])
+    assert_bf16_close(out, ref, "out")
+    inp.residual = np.zeros_like(inp.residual)
+    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "y")
+    dl.close()
+
+
+# --------------------------------------------------------------------------- pinned edge cases
+
+
+def test_seed_is_accumulator_start_on_gpu():
+    """Hand-built layer where seeding decides the result: the GPU gives 0 exactly
+    (seed then ranks), not 2^-24 (routed sum, then shared expert)."""
+    from test_oracle import _seed_counterexample_inputs
+    li = _seed_counterexample_inputs()
+    dl = DeviceLayer(li)
+    out = dl.run(li.x, li.residual)
+    assert oracle.bf16_to_f64(out)[0, 0] == 0.0
+    assert np.array_equal(out, oracle.layer(li))
+    dl.close()
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 5])
+def test_zero_input_leaves_residual_bit_exact(cfg):
+    c = synth.scaled_config(cfg, H=256, I=256) if cfg != 5 else synth.scaled_config(5, H=256, I=256, E=4)
+    inp = synth.make_inputs(c, 3, 0)
+    inp.x = np.zeros_like(inp.x)
+    dl = DeviceLayer(inp)
+    assert np.array_equal(dl.run(inp.x, inp.residual), inp.residual)
+
+
+def test_zero_input_qwen_moe_bit_exact():
+    c = synth.scaled_config(4, H=256, I=64, E=16, k=8, I_s=64)
+    inp = synth.make_inputs(c, 3, 0)
+    inp.x = np.zeros_like(inp.x)
+    dl = DeviceLayer(inp)
+    out, idx = dl.run(inp.x, inp.residual, topk_out=True)
+    assert np.array_equal(idx, np.tile(np.arange(8), (3, 1)))
+    assert np.array_equal(out, inp.residual)
+    dl.close()
+
+
+def test_zero_input_shared_expert_gives_zero():
+    c = synth.scaled_config(3, H=256, I=256)
+    inp = synth.make_inputs(c, 2, 0)
+    inp.x = np.zeros_like(inp.x)
+    assert not np.any(oracle.bf16_to_f64(DeviceLayer(inp).run(inp.x, inp.residual)))
+
+
+def test_moe_single_expert_equals_dense():
+    c = synth.scaled_config(5, H=256, I=320, E=1, k=1)
+    inp = synth.make_inputs(c, 4, 5)
+    moe = DeviceLayer(inp).run(inp.x, inp.residual)
+    ffn = lib.upload_ffn(inp.experts[0])
+    res = dev_bf16(inp.residual)
+    lib.ffn_dense(ffn, dev_bf16(inp.x), res, "silu")
+    assert_bf16_close(moe, host_bf16(res), "moe vs dense")
+
+
+def test_rows_are_independent():
+    """An M-row call equals M single-row calls (the batched pass is the same function)."""
+    c = synth.scaled_config(4, H=256, I=96, E=16, k=4, I_s=64)
+    inp = synth.make_inputs(c, 5, 4)
+    dl = DeviceLayer(inp)
+    full = dl.run(inp.x, inp.residual)
+    for t in range(5):
+        one = dl.run(inp.x[t:t + 1], inp.residual[t:t + 1])
+        assert_bf16_close(one, full[t:t + 1], f"row {t}")
+    dl.close()
+
+
+def test_workspace_too_small_is_refused():
+    c = synth.scaled_config(2, H=256, I=256)
+    inp = synth.make_inputs(c, 2, 0)
+    dl = DeviceLayer(inp)
+    need = lib.workspace_bytes(lib.KIND_DENSE, 2, 256, 256)
+    ws = lib.alloc_workspace(need - 256)
+    with pytest.raises(lib.MoeffnError) as e:
+        lib.ffn_dense(dl.ffn, dev_bf16(inp.x), dev_bf16(inp.residual), "silu", ws=ws)
+    assert e.value.status == -3
