@@ -9,6 +9,7 @@
 #include "../../include/moeffn.h"
 #include "common.cuh"
 #include "gemv.cuh"
+#include "gemv_tma.cuh"
 #include "prof.cuh"
 #include "route.cuh"
 #include "tail.cuh"
@@ -92,15 +93,46 @@ int rows_per_cta(int rows_total) {
   return std::min(64, std::max(8, r));
 }
 
-// K split of a down projection: slices of at most about 2048 elements, a
-// multiple of 32; every split starts below K.
+// K split of a down projection: slices of at most about 4096 elements, a
+// multiple of 256 (16-byte aligned INT4 scale rows); every split starts below K.
 int down_slice(int K) {
-  const int s = (K + 2047) / 2048;
-  return ((K + s - 1) / s + 31) / 32 * 32;
+  const int s = (K + 4095) / 4096;
+  return ((K + s - 1) / s + 255) / 256 * 256;
 }
 int down_splits(int K) {
   const int ks = down_slice(K);
   return (K + ks - 1) / ks;
+}
+
+// ---- TMA-fed GEMV eligibility and geometry ---------------------------------
+
+constexpr size_t kTmaSmemBudget = 200 * 1024;
+constexpr size_t kTmaXBudget = 72 * 1024;
+
+// The bulk copies need 16-byte aligned rows of codes and (INT4) of scales/mins.
+bool tma_ok(const moeffn_qweight& w) {
+  if (w.format == MOEFFN_Q_INT8_ROW) return true;
+  return w.cols % 256 == 0 && aligned16(w.scale) && aligned16(w.min);
+}
+bool tma_ok(const moeffn_ffn& f) { return tma_ok(f.gate) && tma_ok(f.up) && tma_ok(f.down); }
+
+struct TmaGeom {
+  int tokens, stages, mt;
+  bool ok;
+};
+
+TmaGeom tma_geom(int fmt, int nm, int klen, int want_tokens) {
+  TmaGeom g{};
+  g.mt = want_tokens <= 1 ? 1 : 2;
+  const size_t per_tok = tma_gemv_smem(fmt, nm, klen, 1, 1, 0) - 128;
+  int t = (int)std::max<size_t>(1, kTmaXBudget / std::max<size_t>(per_tok, 1));
+  g.tokens = std::max(1, std::min(want_tokens, t));
+  const size_t base = tma_gemv_smem(fmt, nm, klen, g.tokens, g.mt, 0);
+  const size_t st = tma_gemv_stage_bytes(fmt, nm, klen);
+  const int stages = base + 2 * st <= kTmaSmemBudget ? (int)std::min<size_t>(6, (kTmaSmemBudget - base) / st) : 0;
+  g.stages = stages;
+  g.ok = stages >= 2;
+  return g;
 }
 
 int stage_tokens(int fmt, int klen, int want) {
@@ -212,6 +244,55 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, int act, const DenseWS& w,
                   cudaStream_t s) {
   const int fmt = f.gate.format;
+  const int ks = down_slice(I), splits = down_splits(I);
+  const TmaGeom gu = tma_geom(fmt, 2, H, M);
+  const TmaGeom dn = tma_geom(fmt, 1, ks, M);
+  if (tma_ok(f) && gu.ok && dn.ok) {
+    TmaGemvArgs g{};
+    g.fmt = fmt;
+    g.act = act;
+    g.a0 = to_qw(f.gate);
+    g.a1 = to_qw(f.up);
+    g.N = I;
+    g.K = H;
+    g.x = x;
+    g.ld_x = H;
+    g.M = M;
+    g.topk = 1;
+    g.routed_jobs = 1;
+    g.slots = M;
+    g.out_act = w.acts;
+    g.ks_len = H;
+    g.ctas_per_job = kSMs;
+    g.stage_tokens = gu.tokens;
+    g.stages = gu.stages;
+    {
+      ProfScope ps("gateup_gemv_tma", s);
+      MOEFFN_CHECK_CUDA(launch_tma_gemv(g, 2, gu.mt, 1, 1, s), "gate/up launch");
+    }
+    TmaGemvArgs d{};
+    d.fmt = fmt;
+    d.a0 = to_qw(f.down);
+    d.N = H;
+    d.K = I;
+    d.x = w.acts;
+    d.ld_x = I;
+    d.M = M;
+    d.topk = 1;
+    d.routed_jobs = 1;
+    d.slots = M;
+    d.out_d = w.d;
+    d.ks_len = ks;
+    d.ctas_per_job = std::max(1, kSMs / splits);
+    d.stage_tokens = dn.tokens;
+    d.stages = dn.stages;
+    {
+      ProfScope ps("down_gemv_tma", s);
+      MOEFFN_CHECK_CUDA(launch_tma_gemv(d, 1, dn.mt, splits, 1, s), "down launch");
+    }
+    return MOEFFN_OK;
+  }
+
   GateUpArgs g{};
   g.fmt = fmt;
   g.act = act;
@@ -230,7 +311,6 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     ProfScope ps("gateup_gemv", s);
     MOEFFN_CHECK_CUDA(launch_gateup(g, (I + g.rows_per_cta - 1) / g.rows_per_cta, 1, mt_for(M), s), "gate/up launch");
   }
-
   DownArgs d{};
   d.fmt = fmt;
   d.K = I;
@@ -240,8 +320,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
   d.M = M;
   d.slots = M;
   d.d = w.d;
-  d.ks_len = down_slice(I);
-  const int splits = down_splits(I);
+  d.ks_len = ks;
   d.rows_per_cta = rows_per_cta(H * splits);
   d.stage_tokens = stage_tokens(fmt, d.ks_len, M);
   {
@@ -265,6 +344,7 @@ struct moeffn_moe_plan {
   const uint16_t* w_sg;
   moeffn_ffn shared;
   bool has_shared;
+  bool tma;               // every expert (and the shared one) fits the TMA GEMV
   QW* d_gate = nullptr;   // device tables [E]
   QW* d_up = nullptr;
   QW* d_down = nullptr;
@@ -460,8 +540,8 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   if (desc->shared != nullptr) {
     Is = desc->shared->gate.rows;
     if ((rc = check_ffn(*desc->shared, "shared", H, Is)) != MOEFFN_OK) return rc;
-    if (desc->shared->gate.format != MOEFFN_Q_INT4_AFFINE_G32 && desc->shared->gate.format != MOEFFN_Q_INT8_ROW)
-      return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: shared format");
+    if (desc->shared->gate.format != MOEFFN_Q_INT4_AFFINE_G32)
+      return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: the shared expert must be INT4-affine like the routed ones");
     if (desc->shared_gate == nullptr || desc->shared_gate->q == nullptr || desc->shared_gate->format != MOEFFN_BF16 ||
         desc->shared_gate->cols != H || desc->shared_gate->rows != 1 || !aligned16(desc->shared_gate->q))
       return fail(MOEFFN_ERR_INVALID, "moe_plan_create: shared expert needs a BF16 [1][H] 16-byte aligned shared_gate");
@@ -475,6 +555,9 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   p->router_fmt = desc->router.format;
   p->router = desc->router.q;
   p->has_shared = desc->shared != nullptr;
+  p->tma = true;
+  for (int e = 0; e < E; ++e) p->tma = p->tma && tma_ok(desc->experts[e]);
+  if (p->has_shared) p->tma = p->tma && tma_ok(*desc->shared);
   if (p->has_shared) {
     p->shared = *desc->shared;
     p->w_sg = static_cast<const uint16_t*>(desc->shared_gate->q);
@@ -565,6 +648,77 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   const int routed_jobs = std::min(E, P);
   const int jobs = routed_jobs + (p->has_shared ? 1 : 0);
   const int max_tok = M;  // a token selects an expert at most once
+  const MoeSplit sp = moe_split(Ie, Is);
+  const int splits_r = sp.routed, splits_sh = sp.shared;
+  const int splits = std::max(splits_r, splits_sh);
+  const TmaGeom gu = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, H, max_tok);
+  const TmaGeom dn = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 1, sp.ks_len, max_tok);
+  if (p->tma && gu.ok && dn.ok) {
+    TmaGemvArgs g{};
+    g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
+    g.act = p->act;
+    g.tab0 = p->d_gate;
+    g.tab1 = p->d_up;
+    if (p->has_shared) {
+      g.s0 = to_qw(p->shared.gate);
+      g.s1 = to_qw(p->shared.up);
+      g.Ns = Is;
+      g.Ks = H;
+    }
+    g.N = Ie;
+    g.K = H;
+    g.x = x;
+    g.ld_x = H;
+    g.x_s = x;
+    g.M = M;
+    g.topk = k;
+    g.perm = w.perm;
+    g.offsets = w.offsets;
+    g.union_list = w.union_list;
+    g.n_union = w.n_union;
+    g.routed_jobs = routed_jobs;
+    g.slots = P;
+    g.out_act = w.acts;
+    g.out_act_s = w.acts_s;
+    g.ks_len = H;
+    g.ctas_per_job = std::max(1, kSMs / jobs);
+    g.stage_tokens = gu.tokens;
+    g.stages = gu.stages;
+    {
+      ProfScope ps("phase1_gateup_gemv_tma", s);
+      MOEFFN_CHECK_CUDA(launch_tma_gemv(g, 2, gu.mt, 1, jobs, s), "phase-1 launch");
+    }
+    TmaGemvArgs d{};
+    d.fmt = MOEFFN_Q_INT4_AFFINE_G32;
+    d.tab0 = p->d_down;
+    if (p->has_shared) {
+      d.s0 = to_qw(p->shared.down);
+      d.Ns = H;
+      d.Ks = Is;
+    }
+    d.N = H;
+    d.K = Ie;
+    d.x = w.acts;
+    d.ld_x = Ie;
+    d.x_s = w.acts_s;
+    d.M = M;
+    d.topk = k;
+    d.offsets = w.offsets;
+    d.union_list = w.union_list;
+    d.n_union = w.n_union;
+    d.routed_jobs = routed_jobs;
+    d.slots = P;
+    d.out_d = w.d;
+    d.out_d_s = w.d_s;
+    d.ks_len = sp.ks_len;
+    d.ctas_per_job = std::max(1, kSMs / (jobs * splits));
+    d.stage_tokens = dn.tokens;
+    d.stages = dn.stages;
+    {
+      ProfScope ps("phase2_down_gemv_tma", s);
+      MOEFFN_CHECK_CUDA(launch_tma_gemv(d, 1, dn.mt, splits, jobs, s), "phase-2 launch");
+    }
+  } else {
   GateUpArgs g{};
   g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
   g.act = p->act;
@@ -590,8 +744,6 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   // Expected active rows: min(E, P) experts of Ie rows (+ the shared expert).
   g.rows_per_cta = rows_per_cta(std::min(E, P) * Ie + Is);
   g.stage_tokens = stage_tokens(g.fmt, H, max_tok);
-  if (p->has_shared && p->shared.gate.format != MOEFFN_Q_INT4_AFFINE_G32)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "moe_layer: shared expert must share the routed format");
   const int gx = (std::max(Ie, Is) + g.rows_per_cta - 1) / g.rows_per_cta;
   {
     ProfScope ps("phase1_gateup_gemv", s);
@@ -616,9 +768,7 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   d.d = w.d;
   d.d_s = w.d_s;
   // One slice length for routed and shared jobs; each job has its own count.
-  const MoeSplit sp = moe_split(Ie, Is);
   d.ks_len = sp.ks_len;
-  const int splits_r = sp.routed, splits_sh = sp.shared;
   d.rows_per_cta = rows_per_cta(H * std::max(1, std::min(E, P) / 4));
   d.stage_tokens = stage_tokens(d.fmt, d.ks_len, max_tok);
   {
@@ -626,6 +776,7 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     MOEFFN_CHECK_CUDA(launch_down(d, (H + d.rows_per_cta - 1) / d.rows_per_cta, std::max(splits_r, splits_sh), jobs,
                                   mt_for(std::min(M, 2)), s),
                       "phase-2 launch");
+  }
   }
 
   TailArgs t{};

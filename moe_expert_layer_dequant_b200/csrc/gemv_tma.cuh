@@ -1,0 +1,42 @@
+// Launch interface of the TMA-fed GEMV (gemv_tma.cu).
+#pragma once
+#include "common.cuh"
+
+namespace moeffn {
+
+constexpr int kTmaConsumers = 8;  // consumer warps per CTA = rows per stage
+
+struct TmaGemvArgs {
+  int fmt, act;
+  QW a0, a1;                   // dense mode: matrices (a1: up, when fused)
+  const QW* tab0;              // grouped mode: per-expert tables (device)
+  const QW* tab1;
+  QW s0, s1;                   // shared expert matrices
+  int N, K;                    // dense / routed rows and reduction width
+  int Ns, Ks;                  // shared rows and width
+  const uint16_t* x;           // dense / routed input rows
+  int ld_x;                    // row stride of x (elements)
+  const uint16_t* x_s;         // shared job input rows (row stride Ks)
+  int M, topk;
+  const int* perm;             // routed gate/up: input row of slot s = perm[s] / topk
+  const int* offsets;          // null: dense mode
+  const int* union_list;
+  const int* n_union;
+  int routed_jobs;
+  int slots;                   // slot count of out_d (dense: M, routed: M*topk)
+  uint16_t* out_act;           // fused gate/up: [slots][N] bf16
+  uint16_t* out_act_s;         // [M][Ns]
+  float* out_d;                // down: [splits][slots][N] fp32 partial sums
+  float* out_d_s;              // [splits][M][N]
+  int ks_len;                  // K elements per split (INT4: multiple of 256)
+  int ctas_per_job;
+  int stage_tokens;
+  int stages;
+};
+
+size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages);
+size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
+cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, int jobs, cudaStream_t s);
+unsigned int tma_gemv_fault_flags(bool clear);
+
+}  // namespace moeffn

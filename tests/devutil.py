@@ -23,14 +23,37 @@ def rms(v: np.ndarray) -> float:
     return float(np.sqrt(np.mean(np.asarray(v, np.float64) ** 2)))
 
 
+def bf16_ulp(v: np.ndarray) -> np.ndarray:
+    """Spacing of bf16 numbers at |v| (8 significant bits)."""
+    a = np.maximum(np.abs(np.asarray(v, np.float64)), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(a)) - 7)
+
+
 def assert_bf16_close(got_bits: np.ndarray, want_bits: np.ndarray, what: str = "", rtol: float = RTOL_RMS):
+    """max |got - want| <= rtol * RMS(want) on bf16 outputs, up to rounding flips.
+
+    Both sides round their own pre-rounding values (fp32 here, float64 in the
+    oracle) to bf16 wherever the layer stores a 2-byte value, the output being
+    the last. Where the two straddle a rounding boundary the stored values
+    differ by one bf16 ulp, and a flip in a stored intermediate (h1 before the
+    norm, the activation) can add one more. For |v| >= 2.56 * RMS one ulp
+    already exceeds 2e-2 * RMS, so an element may instead differ by at most
+    two bf16 ulps of its magnitude; such elements must be rare (< 1%).
+    """
     g = oracle.bf16_to_f64(got_bits)
     w = oracle.bf16_to_f64(want_bits)
     assert g.shape == w.shape, (g.shape, w.shape)
     scale = rms(w)
-    err = float(np.max(np.abs(g - w))) if g.size else 0.0
-    assert err <= rtol * max(scale, 1e-30), f"{what}: max|err| {err:.3e} > {rtol} * RMS {scale:.3e}"
-    return err / max(scale, 1e-30)
+    if g.size == 0:
+        return 0.0
+    err = np.abs(g - w)
+    tol = rtol * max(scale, 1e-30)
+    flip = (err > tol) & (err <= 2 * bf16_ulp(np.maximum(np.abs(g), np.abs(w))))
+    bad = (err > tol) & ~flip
+    worst = float(np.max(np.where(flip, 0.0, err)))
+    assert not np.any(bad), f"{what}: max|err| {float(err[bad].max()):.3e} > {rtol} * RMS {scale:.3e} ({int(bad.sum())} elements)"
+    assert flip.mean() < 1e-2, f"{what}: {int(flip.sum())} rounding flips of {g.size}"
+    return worst / max(scale, 1e-30)
 
 
 class DeviceLayer:

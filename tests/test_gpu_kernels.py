@@ -103,8 +103,10 @@ def test_router_logits_and_topk_end_to_end():
 
 
 DENSE_SMALL = [
-    (1, dict(H=256, I=416), FMT_INT8_ROW),
-    (2, dict(H=640, I=1056), FMT_INT4_G32),
+    (1, dict(H=256, I=416), FMT_INT8_ROW),      # bulk-copy GEMV (INT8 rows)
+    (2, dict(H=640, I=1056), FMT_INT4_G32),     # K % 256 != 0: register-load GEMV
+    (2, dict(H=512, I=1280), FMT_INT4_G32),     # bulk-copy GEMV, ragged CTA row ranges
+    (2, dict(H=256, I=4352), FMT_INT4_G32),     # down split along K: per-row bulk copies
 ]
 
 
@@ -129,9 +131,12 @@ def test_shared_expert_small(M):
 
 
 MOE_SMALL = [
-    dict(cfg=4, H=256, I=96, E=16, k=4, I_s=64),
+    dict(cfg=4, H=256, I=96, E=16, k=4, I_s=64),     # register-load GEMV path
     dict(cfg=5, H=320, I=192, E=8, k=2, I_s=0),
     dict(cfg=4, H=256, I=64, E=4, k=4, I_s=128),
+    dict(cfg=4, H=512, I=256, E=16, k=4, I_s=256),   # bulk-copy GEMV path
+    dict(cfg=5, H=768, I=512, E=8, k=2, I_s=0),
+    dict(cfg=5, H=256, I=4608, E=4, k=2, I_s=0),     # expert down split along K
 ]
 
 
