@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "gemv.cuh"
 #include "gemv_tma.cuh"
+#include "tmap.cuh"
 #include "prof.cuh"
 #include "route.cuh"
 #include "tail.cuh"
@@ -93,15 +94,21 @@ int rows_per_cta(int rows_total) {
   return std::min(64, std::max(8, r));
 }
 
-// K split of a down projection: slices of at most about 4096 elements, a
-// multiple of 256 (16-byte aligned INT4 scale rows); every split starts below K.
-int down_slice(int K) {
-  const int s = (K + 4095) / 4096;
+// K split of a down projection: slices of at most 4096 (INT4) or 2048 (INT8)
+// elements, a multiple of 256 (16-byte aligned scale rows and TMA boxes of at
+// most 256 eight-byte elements); every split starts below K.
+int down_slice(int K, int fmt) {
+  const int lim = fmt == MOEFFN_Q_INT8_ROW ? 2048 : 4096;
+  const int s = (K + lim - 1) / lim;
   return ((K + s - 1) / s + 255) / 256 * 256;
 }
-int down_splits(int K) {
-  const int ks = down_slice(K);
+int down_splits(int K, int fmt) {
+  const int ks = down_slice(K, fmt);
   return (K + ks - 1) / ks;
+}
+// Partial-sum buffers are sized for the format with more splits.
+int down_splits_any(int K) {
+  return std::max(down_splits(K, MOEFFN_Q_INT8_ROW), down_splits(K, MOEFFN_Q_INT4_AFFINE_G32));
 }
 
 // ---- TMA-fed GEMV eligibility and geometry ---------------------------------
@@ -164,7 +171,7 @@ struct DenseWS {
 DenseWS carve_dense(Carve& c, int M, int H, int I) {
   DenseWS w;
   w.acts = c.take<uint16_t>((size_t)M * I);
-  w.d = c.take<float>((size_t)down_splits(I) * M * H);
+  w.d = c.take<float>((size_t)down_splits_any(I) * M * H);
   return w;
 }
 
@@ -191,7 +198,7 @@ struct MoeSplit {
 
 MoeSplit moe_split(int Ie, int Is) {
   MoeSplit s;
-  s.ks_len = down_slice(std::max(Ie, Is));
+  s.ks_len = down_slice(std::max(Ie, Is), MOEFFN_Q_INT4_AFFINE_G32);
   s.routed = (Ie + s.ks_len - 1) / s.ks_len;
   s.shared = Is > 0 ? (Is + s.ks_len - 1) / s.ks_len : 0;
   return s;
@@ -244,7 +251,7 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, int act, const DenseWS& w,
                   cudaStream_t s) {
   const int fmt = f.gate.format;
-  const int ks = down_slice(I), splits = down_splits(I);
+  const int ks = down_slice(I, fmt), splits = down_splits(I, fmt);
   const TmaGeom gu = tma_geom(fmt, 2, H, M);
   const TmaGeom dn = tma_geom(fmt, 1, ks, M);
   if (tma_ok(f) && gu.ok && dn.ok) {
@@ -283,6 +290,8 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.slots = M;
     d.out_d = w.d;
     d.ks_len = ks;
+    d.use_maps = splits > 1;
+    if (d.use_maps) MOEFFN_CHECK_CUDA(encode_qw_maps(&d.dmap, fmt, to_qw(f.down), H, I, ks), "tensor map encode");
     d.ctas_per_job = std::max(1, kSMs / splits);
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;
@@ -348,6 +357,8 @@ struct moeffn_moe_plan {
   QW* d_gate = nullptr;   // device tables [E]
   QW* d_up = nullptr;
   QW* d_down = nullptr;
+  QWMaps* d_maps = nullptr;    // [E] tensor maps of the expert down matrices (K split)
+  QWMaps* d_maps_s = nullptr;  // [1] shared expert down (K split)
 };
 
 extern "C" {
@@ -387,7 +398,7 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
   if (rc != MOEFFN_OK) return rc;
   if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "ffn_dense: x/residual not 16-byte aligned");
   if (x == residual) return fail(MOEFFN_ERR_INVALID, "ffn_dense: x aliases residual");
-  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax || gemv_stage_bytes(w->gate.format, down_slice(I), 1) > kStageMax)
+  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax || gemv_stage_bytes(w->gate.format, down_slice(I, w->gate.format), 1) > kStageMax)
     return fail(MOEFFN_ERR_UNSUPPORTED, "ffn_dense: hidden size %d too large for the staged GEMV", H);
   Carve c{nullptr};
   carve_dense(c, M, H, I);
@@ -401,7 +412,7 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
   t.M = M;
   t.N = H;
   t.d = d.d;
-  t.splits = down_splits(I);
+  t.splits = down_splits(I, w->gate.format);
   t.slots = M;
   t.res = residual;
   {
@@ -439,7 +450,7 @@ int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* no
   t.M = M;
   t.N = H;
   t.d = d.d;
-  t.splits = down_splits(I);
+  t.splits = down_splits(I, w->gate.format);
   t.slots = M;
   t.h1 = h1_out;
   t.norm_w = norm_w;
@@ -576,6 +587,28 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
     moe_plan_destroy(p);
     return fail(MOEFFN_ERR_CUDA, "moe_plan_create: copy of the pointer tables failed");
   }
+  // Tensor maps for the down projections split along K (bulk-copy GEMV).
+  const MoeSplit sp = moe_split(Ie, Is);
+  if (p->tma && (sp.routed > 1 || sp.shared > 1)) {
+    std::vector<QWMaps> maps(E);
+    bool ok = true;
+    for (int e = 0; e < E && ok; ++e)
+      ok = encode_qw_maps(&maps[e], MOEFFN_Q_INT4_AFFINE_G32, d[e], H, Ie, sp.ks_len) == cudaSuccess;
+    QWMaps ms{};
+    if (ok && p->has_shared && sp.shared > 1)
+      ok = encode_qw_maps(&ms, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.down), H, Is, sp.ks_len) == cudaSuccess;
+    if (!ok) {
+      moe_plan_destroy(p);
+      return fail(MOEFFN_ERR_CUDA, "moe_plan_create: tensor map encoding failed");
+    }
+    if (cudaMalloc(&p->d_maps, sizeof(QWMaps) * E) != cudaSuccess ||
+        cudaMemcpy(p->d_maps, maps.data(), sizeof(QWMaps) * E, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMalloc(&p->d_maps_s, sizeof(QWMaps)) != cudaSuccess ||
+        cudaMemcpy(p->d_maps_s, &ms, sizeof(QWMaps), cudaMemcpyHostToDevice) != cudaSuccess) {
+      moe_plan_destroy(p);
+      return fail(MOEFFN_ERR_CUDA, "moe_plan_create: tensor map upload failed");
+    }
+  }
   *plan = p;
   return MOEFFN_OK;
 }
@@ -585,6 +618,8 @@ int moe_plan_destroy(moeffn_moe_plan* plan) {
   cudaFree(plan->d_gate);
   cudaFree(plan->d_up);
   cudaFree(plan->d_down);
+  cudaFree(plan->d_maps);
+  cudaFree(plan->d_maps_s);
   delete plan;
   return MOEFFN_OK;
 }
@@ -711,6 +746,9 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     d.out_d = w.d;
     d.out_d_s = w.d_s;
     d.ks_len = sp.ks_len;
+    d.use_maps = splits > 1;
+    d.maps = p->d_maps;
+    d.maps_s = p->d_maps_s;
     d.ctas_per_job = std::max(1, kSMs / (jobs * splits));
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;

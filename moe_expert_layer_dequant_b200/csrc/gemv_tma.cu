@@ -20,64 +20,80 @@
 // A CTA takes a contiguous range of the job's rows (a multiple of R rows).
 #include "gemv_tma.cuh"
 #include "sync.cuh"
+#include "tmap.cuh"
 
 namespace moeffn {
 
 namespace {
 
+// Activations are staged per 16-byte weight chunk as int16 fixed point with one
+// power-of-two factor per chunk: x = xi * 2^(e-14), e = floor(log2(max|x|)).
+// A bf16 value has 8 significant bits, so every value within 2^7 of the
+// chunk's largest is exact and the rest lose only bits below 2^(e-15).
+// Codes times xi are then summed exactly in int32 with DP2A (two 16x8-bit
+// products per instruction) and scaled once per chunk.
+__device__ __forceinline__ int dp2a_lo_u(int a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi_u(int a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_lo_s(int a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ int dp2a_hi_s(int a, uint32_t b, int c) {
+  int d;
+  asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
 template <int FMT>
 struct Codes;
 
+// INT4: a chunk is one group of 32 codes (4 words). Word codes q0..q7: the
+// low nibbles of its bytes are q0,q2,q4,q6 and the high nibbles q1,q3,q5,q7,
+// so the staged int16 of a word are ordered x0,x2,x4,x6,x1,x3,x5,x7.
 template <>
 struct Codes<FMT_INT4_G32> {
-  static constexpr int kChunk = 32;      // codes per 16-byte chunk (one group)
-  static constexpr int kStride = 36;     // padded fp32 stride of a staged chunk
-  static constexpr int kFloat2 = 4;      // float2 per 32-bit word
-  static __device__ __forceinline__ float pos_scale(int k) { return int4_pos_scale(k); }
-  // Positioned codes q_i * 16^(i%4) of one word: one LOP3 per code.
-  static __device__ __forceinline__ void word(uint32_t w, float2 (&c)[4]) {
-    const uint32_t hi = w >> 16;
-    const uint32_t m0 = 0x000Fu, m1 = 0x00F0u, m2 = 0x0F00u, m3 = 0xF000u, mg = kMagic;
-    float2 a, b, d, e;
-    a.x = __uint_as_float(and_or(w, m0, mg));
-    a.y = __uint_as_float(and_or(w, m1, mg));
-    b.x = __uint_as_float(and_or(w, m2, mg));
-    b.y = __uint_as_float(and_or(w, m3, mg));
-    d.x = __uint_as_float(and_or(hi, m0, mg));
-    d.y = __uint_as_float(and_or(hi, m1, mg));
-    e.x = __uint_as_float(and_or(hi, m2, mg));
-    e.y = __uint_as_float(and_or(hi, m3, mg));
-    const float2 sub = make_float2(-kMagicF, -kMagicF);
-    c[0] = __fadd2_rn(a, sub);
-    c[1] = __fadd2_rn(b, sub);
-    c[2] = __fadd2_rn(d, sub);
-    c[3] = __fadd2_rn(e, sub);
+  static constexpr int kChunk = 32;
+  static constexpr int kStageBytes = 80;  // 64 bytes of int16 + 16 bytes pad (bank spread)
+  static __device__ __forceinline__ int slot_of(int j) {  // position of element j of a word
+    return (j & 1) * 4 + (j >> 1);
+  }
+  // Adds the 8 products of word w with its staged activations (16 bytes).
+  static __device__ __forceinline__ void dot_word(uint32_t w, uint4 x, int& p0, int& p1) {
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    p0 = dp2a_lo_u((int)x.x, lo, p0);
+    p1 = dp2a_hi_u((int)x.y, lo, p1);
+    p0 = dp2a_lo_u((int)x.z, hi, p0);
+    p1 = dp2a_hi_u((int)x.w, hi, p1);
   }
 };
 
+// INT8: a chunk is 16 signed codes (4 words); staged in natural order.
 template <>
 struct Codes<FMT_INT8_ROW> {
   static constexpr int kChunk = 16;
-  static constexpr int kStride = 20;
-  static constexpr int kFloat2 = 2;
-  static __device__ __forceinline__ float pos_scale(int k) { return int8_pos_scale(k); }
-  static __device__ __forceinline__ void word(uint32_t w, float2 (&c)[4]) {
-    const uint32_t hi = w >> 16;
-    const uint32_t m0 = 0x00FFu, m1 = 0xFF00u, x0 = 0x0080u | kMagic, x1 = 0x8000u | kMagic;
-    float2 a, b;
-    a.x = __uint_as_float(and_xor(w, m0, x0));
-    a.y = __uint_as_float(and_xor(w, m1, x1));
-    b.x = __uint_as_float(and_xor(hi, m0, x0));
-    b.y = __uint_as_float(and_xor(hi, m1, x1));
-    const float2 sub = make_float2(-(kMagicF + 128.0f), -(kMagicF + 32768.0f));
-    c[0] = __fadd2_rn(a, sub);
-    c[1] = __fadd2_rn(b, sub);
+  static constexpr int kStageBytes = 48;  // 32 bytes of int16 + 16 bytes pad
+  static __device__ __forceinline__ int slot_of(int j) { return j; }
+  // Two words (8 codes) with their staged activations (16 bytes).
+  static __device__ __forceinline__ void dot_word(uint32_t w0, uint32_t w1, uint4 x, int& p0, int& p1) {
+    p0 = dp2a_lo_s((int)x.x, w0, p0);
+    p1 = dp2a_hi_s((int)x.y, w0, p1);
+    p0 = dp2a_lo_s((int)x.z, w1, p0);
+    p1 = dp2a_hi_s((int)x.w, w1, p1);
   }
 };
 
 struct Job {
   QW m[2];
-  int N, K, ntok, slot0;
+  int N, K, ntok, slot0, expert;
   bool gather, shared, valid;
 };
 
@@ -90,6 +106,7 @@ __device__ __forceinline__ Job decode_job(const TmaGemvArgs& a) {
   } else if (z < a.routed_jobs) {
     if (z >= *a.n_union) { j.valid = false; return j; }
     const int e = a.union_list[z];
+    j.expert = e;
     j.m[0] = a.tab0[e];
     if (a.tab1 != nullptr) j.m[1] = a.tab1[e];
     j.N = a.N; j.K = a.K;
@@ -107,7 +124,7 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 }
 
 template <int FMT, int MT, int NM, int NC>
-__global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const TmaGemvArgs a) {
+__global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_constant__ TmaGemvArgs a) {
   using C = Codes<FMT>;
   constexpr bool kInt4 = (FMT == FMT_INT4_G32);
   constexpr int R = NC;  // rows per stage: one per consumer warp
@@ -122,22 +139,31 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const TmaGemvArgs
   const int r0 = blockIdx.x * rpc;
   const int r1 = min(job.N, r0 + rpc);
   if (r0 >= r1) return;
+  // A job split along K loads boxes through its tensor maps; an unsplit job
+  // copies whole (contiguous) rows.
+  const bool maps = a.use_maps != 0 && job.K > a.ks_len;
+  const QWMaps* jm = nullptr;
+  if (maps) jm = a.offsets == nullptr ? &a.dmap : (job.shared ? a.maps_s : a.maps + job.expert);
 
   // ---- shared memory carve ------------------------------------------------
+  // Stage rows are `cs` code bytes and `gst` groups apart: the full box width
+  // (ks_len) with tensor maps, the slice itself with 1-D copies.
   const int S = a.stages;
-  const int cb = kInt4 ? klen / 2 : klen;        // code bytes per row
-  const int gs = kInt4 ? klen / 32 : 0;          // groups per row
+  const int wid = maps ? a.ks_len : klen;
+  const int cs = kInt4 ? wid / 2 : wid;
+  const int gst = kInt4 ? wid / 32 : 0;
   const int nch = klen / C::kChunk;
-  const int tok_stride = nch * C::kStride;
+  const int tok_stride = nch * C::kStageBytes;   // bytes of staged int16 per token
   const int tok_rows = (a.stage_tokens + MT - 1) / MT * MT;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + S;
-  float* xs = reinterpret_cast<float*>(smem + 128);
-  float* xsum = xs + tok_rows * tok_stride;
-  const size_t x_bytes = ((size_t)tok_rows * (tok_stride + gs) * 4 + 127) / 128 * 128;
+  uint8_t* xi = smem + 128;                                         // [tok_rows][nch] chunks
+  float* xf = reinterpret_cast<float*>(xi + (size_t)tok_rows * tok_stride);  // [tok_rows][nch] factors
+  float* xsum = xf + (size_t)tok_rows * nch;                        // [tok_rows][nch] (INT4)
+  const size_t x_bytes = ((size_t)tok_rows * (tok_stride + 4 * nch + (kInt4 ? 4 * nch : 0)) + 127) / 128 * 128;
   uint8_t* stage0 = smem + 128 + x_bytes;
-  const size_t stage_bytes = (size_t)NM * R * (cb + 4 * gs);
-  // within a stage: codes [NM][R][cb], scales [NM][R][gs], mins [NM][R][gs]
+  const size_t stage_bytes = (size_t)NM * R * (cs + 4 * gst);
+  // within a stage: codes [NM][R][cs], scales [NM][R][gst], mins [NM][R][gst]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -164,29 +190,31 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const TmaGemvArgs
         const int n0 = r0 + (s % row_stages) * R;
         const int nr = min(R, r1 - n0);
         uint8_t* st = stage0 + (size_t)slot * stage_bytes;
-        mbar_arrive_expect_tx(&full[slot], (uint32_t)(NM * nr * (cb + 4 * gs)));
+        uint8_t* dsc = st + (size_t)NM * R * cs;
+        uint8_t* dmn = dsc + (size_t)NM * R * gst * 2;
+        if (maps) {
+          // Whole boxes: rows past the end of the matrix arrive as zeros.
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)stage_bytes);
 #pragma unroll
-        for (int i = 0; i < NM; ++i) {
-          const uint8_t* q = job.m[i].q + (size_t)n0 * row_bytes + (kInt4 ? k0 / 2 : k0);
-          uint8_t* dq = st + (size_t)i * R * cb;
-          if (klen == job.K) {
-            bulk_g2s(dq, q, (uint32_t)(nr * cb), &full[slot]);
-          } else {
-            for (int r = 0; r < nr; ++r) bulk_g2s(dq + r * cb, q + (size_t)r * row_bytes, cb, &full[slot]);
+          for (int i = 0; i < NM; ++i) {
+            tma_load_2d(st + (size_t)i * R * cs, &jm[i].codes, kInt4 ? k0 / 16 : k0 / 8, n0, &full[slot]);
+            if (kInt4) {
+              tma_load_2d(dsc + (size_t)i * R * gst * 2, &jm[i].scale, k0 / 32, n0, &full[slot]);
+              tma_load_2d(dmn + (size_t)i * R * gst * 2, &jm[i].mn, k0 / 32, n0, &full[slot]);
+            }
           }
-          if (kInt4) {
-            const uint8_t* sc = reinterpret_cast<const uint8_t*>(job.m[i].scale) + ((size_t)n0 * row_groups + k0 / 32) * 2;
-            const uint8_t* mn = reinterpret_cast<const uint8_t*>(job.m[i].mn) + ((size_t)n0 * row_groups + k0 / 32) * 2;
-            uint8_t* ds = st + (size_t)NM * R * cb + (size_t)i * R * gs * 2;
-            uint8_t* dm = st + (size_t)NM * R * cb + (size_t)NM * R * gs * 2 + (size_t)i * R * gs * 2;
-            if (klen == job.K) {
-              bulk_g2s(ds, sc, (uint32_t)(nr * gs * 2), &full[slot]);
-              bulk_g2s(dm, mn, (uint32_t)(nr * gs * 2), &full[slot]);
-            } else {
-              for (int r = 0; r < nr; ++r) {
-                bulk_g2s(ds + r * gs * 2, sc + (size_t)r * row_groups * 2, gs * 2, &full[slot]);
-                bulk_g2s(dm + r * gs * 2, mn + (size_t)r * row_groups * 2, gs * 2, &full[slot]);
-              }
+        } else {
+          // Whole rows are contiguous: one copy per array for the stage.
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)(NM * nr * (cs + 4 * gst)));
+#pragma unroll
+          for (int i = 0; i < NM; ++i) {
+            bulk_g2s(st + (size_t)i * R * cs, job.m[i].q + (size_t)n0 * row_bytes, (uint32_t)(nr * cs), &full[slot]);
+            if (kInt4) {
+              const size_t go = (size_t)n0 * row_groups * 2;
+              bulk_g2s(dsc + (size_t)i * R * gst * 2, reinterpret_cast<const uint8_t*>(job.m[i].scale) + go,
+                       (uint32_t)(nr * gst * 2), &full[slot]);
+              bulk_g2s(dmn + (size_t)i * R * gst * 2, reinterpret_cast<const uint8_t*>(job.m[i].mn) + go,
+                       (uint32_t)(nr * gst * 2), &full[slot]);
             }
           }
         }
@@ -204,48 +232,50 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const TmaGemvArgs
   for (int tb = 0; tb < job.ntok; tb += a.stage_tokens) {
     const int tn = min(a.stage_tokens, job.ntok - tb);
     consumer_sync(nthreads);
-    // Stage token rows tb..tb+tn (K slice) as position-scaled fp32; zero pad rows.
-    const int per_row = klen / 8;
-    for (int i = threadIdx.x; i < tok_rows * per_row; i += nthreads) {
-      const int r = i / per_row;
-      const int kk = (i - r * per_row) * 8;
-      float f[8];
+    // Stage token rows tb..tb+tn (K slice) chunk by chunk: int16 fixed point,
+    // the chunk's power-of-two factor and (INT4) its plain sum; zero pad rows.
+    for (int i = threadIdx.x; i < tok_rows * nch; i += nthreads) {
+      const int r = i / nch, c = i - r * nch;
+      uint16_t v[C::kChunk];
       if (r < tn) {
         const int row = job.gather ? a.perm[job.slot0 + tb + r] / a.topk : job.slot0 + tb + r;
-        const uint4 v = *reinterpret_cast<const uint4*>(src + (size_t)row * ld + k0 + kk);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)row * ld + k0 + c * C::kChunk);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          f[2 * j] = __uint_as_float(w[j] << 16) * C::pos_scale(kk + 2 * j);
-          f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u) * C::pos_scale(kk + 2 * j + 1);
+        for (int q = 0; q < C::kChunk / 8; ++q) {
+          const uint4 u = p[q];
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            v[8 * q + 2 * j] = (uint16_t)(w[j] & 0xFFFFu);
+            v[8 * q + 2 * j + 1] = (uint16_t)(w[j] >> 16);
+          }
         }
       } else {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] = 0.f;
+        for (int j = 0; j < C::kChunk; ++j) v[j] = 0;
       }
-      const int c = kk / C::kChunk, o = kk - c * C::kChunk;
-      float* dst = xs + r * tok_stride + c * C::kStride + o;
-      *reinterpret_cast<float4*>(dst) = make_float4(f[0], f[1], f[2], f[3]);
-      *reinterpret_cast<float4*>(dst + 4) = make_float4(f[4], f[5], f[6], f[7]);
-    }
-    if (kInt4) {
-      const int gsd = gs > 0 ? gs : 1;
-      for (int i = threadIdx.x; i < tok_rows * gs; i += nthreads) {
-        const int r = i / gsd, g = i - r * gsd;
-        float sum = 0.f;
-        if (r < tn) {
-          const int row = job.gather ? a.perm[job.slot0 + tb + r] / a.topk : job.slot0 + tb + r;
-          const uint16_t* p = src + (size_t)row * ld + k0 + g * 32;
+      float amax = 0.f, sum = 0.f;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 v = *reinterpret_cast<const uint4*>(p + 8 * q);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) sum += __uint_as_float(w[j] << 16) + __uint_as_float(w[j] & 0xFFFF0000u);
-          }
-        }
-        xsum[r * gs + g] = sum;
+      for (int j = 0; j < C::kChunk; ++j) {
+        const float f = bf16_bits_to_float(v[j]);
+        amax = fmaxf(amax, fabsf(f));
+        sum += f;
       }
+      int e = 0;
+      if (amax > 0.f) {
+        frexpf(amax, &e);
+        e -= 1;                                   // amax in [2^e, 2^(e+1))
+      }
+      int16_t* dst = reinterpret_cast<int16_t*>(xi + (size_t)r * tok_stride + c * C::kStageBytes);
+#pragma unroll
+      for (int j = 0; j < C::kChunk; ++j) {
+        const float f = bf16_bits_to_float(v[j]);
+        const int word = j / (C::kChunk == 32 ? 8 : 4), pos = j % (C::kChunk == 32 ? 8 : 4);
+        dst[word * (C::kChunk == 32 ? 8 : 4) + C::slot_of(pos)] =
+            (int16_t)(amax > 0.f ? __float2int_rn(ldexpf(f, 14 - e)) : 0);
+      }
+      xf[r * nch + c] = amax > 0.f ? ldexpf(1.0f, e - 14) : 0.f;
+      if (kInt4) xsum[r * nch + c] = sum;
     }
     consumer_sync(nthreads);
 
@@ -267,10 +297,10 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const TmaGemvArgs
         const __half* mns[NM];
 #pragma unroll
         for (int i = 0; i < NM; ++i) {
-          codes[i] = st + ((size_t)i * R + warp) * cb;
-          scl[i] = reinterpret_cast<const __half*>(st + (size_t)NM * R * cb) + ((size_t)i * R + warp) * gs;
-          mns[i] = reinterpret_cast<const __half*>(st + (size_t)NM * R * cb + (size_t)NM * R * gs * 2) +
-                   ((size_t)i * R + warp) * gs;
+          codes[i] = st + ((size_t)i * R + warp) * cs + lane * 16;
+          scl[i] = reinterpret_cast<const __half*>(st + (size_t)NM * R * cs) + ((size_t)i * R + warp) * gst + lane;
+          mns[i] = reinterpret_cast<const __half*>(st + (size_t)NM * R * cs + (size_t)NM * R * gst * 2) +
+                   ((size_t)i * R + warp) * gst + lane;
         }
         for (int tc = 0; tc < tn; tc += MT) {
           float acc[NM][MT];
@@ -278,55 +308,62 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const TmaGemvArgs
           for (int i = 0; i < NM; ++i)
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[i][t] = 0.f;
-          const float* xb = xs + tc * tok_stride;
-          for (int c = lane; c < nch; c += 32) {
+          const uint8_t* xl = xi + (size_t)tc * tok_stride + lane * C::kStageBytes;
+          const int iters = (nch - lane + 31) >> 5;
+          for (int it = 0; it < iters; ++it) {
+            const int c = lane + 32 * it;
             uint4 wv[NM];
             float sc[NM], mn[NM];
 #pragma unroll
             for (int i = 0; i < NM; ++i) {
-              wv[i] = *reinterpret_cast<const uint4*>(codes[i] + c * 16);
+              wv[i] = *reinterpret_cast<const uint4*>(codes[i] + it * 512);
               if (kInt4) {
-                sc[i] = __half2float(scl[i][c]);
-                mn[i] = __half2float(mns[i][c]);
+                sc[i] = __half2float(scl[i][it * 32]);
+                mn[i] = __half2float(mns[i][it * 32]);
               }
             }
-            float2 p[NM][MT];
+            const uint8_t* xc = xl + it * 32 * C::kStageBytes;
+            int p0[NM][MT], p1[NM][MT];
 #pragma unroll
             for (int i = 0; i < NM; ++i)
 #pragma unroll
-              for (int t = 0; t < MT; ++t) p[i][t] = make_float2(0.f, 0.f);
+              for (int t = 0; t < MT; ++t) p0[i][t] = p1[i][t] = 0;
+            if (kInt4) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float2 cf[NM][4];
+              for (int q = 0; q < 4; ++q) {
 #pragma unroll
-              for (int i = 0; i < NM; ++i) {
-                const uint32_t w = q == 0 ? wv[i].x : q == 1 ? wv[i].y : q == 2 ? wv[i].z : wv[i].w;
-                C::word(w, cf[i]);
+                for (int t = 0; t < MT; ++t) {
+                  const uint4 x4 = *reinterpret_cast<const uint4*>(xc + (size_t)t * tok_stride + q * 16);
+#pragma unroll
+                  for (int i = 0; i < NM; ++i) {
+                    const uint32_t w = q == 0 ? wv[i].x : q == 1 ? wv[i].y : q == 2 ? wv[i].z : wv[i].w;
+                    Codes<FMT_INT4_G32>::dot_word(w, x4, p0[i][t], p1[i][t]);
+                  }
+                }
               }
+            } else {
 #pragma unroll
-              for (int t = 0; t < MT; ++t) {
-                const float* xp = xb + t * tok_stride + c * C::kStride + q * 2 * C::kFloat2;
-                const float4 xa = *reinterpret_cast<const float4*>(xp);
-                float4 xc = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (C::kFloat2 == 4) xc = *reinterpret_cast<const float4*>(xp + 4);
+              for (int h = 0; h < 2; ++h) {
 #pragma unroll
-                for (int i = 0; i < NM; ++i) {
-                  p[i][t] = __ffma2_rn(cf[i][0], make_float2(xa.x, xa.y), p[i][t]);
-                  p[i][t] = __ffma2_rn(cf[i][1], make_float2(xa.z, xa.w), p[i][t]);
-                  if (C::kFloat2 == 4) {
-                    p[i][t] = __ffma2_rn(cf[i][2], make_float2(xc.x, xc.y), p[i][t]);
-                    p[i][t] = __ffma2_rn(cf[i][3], make_float2(xc.z, xc.w), p[i][t]);
+                for (int t = 0; t < MT; ++t) {
+                  const uint4 x4 = *reinterpret_cast<const uint4*>(xc + (size_t)t * tok_stride + h * 16);
+#pragma unroll
+                  for (int i = 0; i < NM; ++i) {
+                    const uint32_t w0 = h == 0 ? wv[i].x : wv[i].z, w1 = h == 0 ? wv[i].y : wv[i].w;
+                    Codes<FMT_INT8_ROW>::dot_word(w0, w1, x4, p0[i][t], p1[i][t]);
                   }
                 }
               }
             }
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-              const float X = kInt4 ? xsum[(tc + t) * gs + c] : 0.f;
+              const float f = xf[(tc + t) * nch + c];
+              const float X = kInt4 ? xsum[(tc + t) * nch + c] : 0.f;
 #pragma unroll
               for (int i = 0; i < NM; ++i) {
-                const float P = p[i][t].x + p[i][t].y;
-                acc[i][t] = kInt4 ? fmaf(sc[i], P, fmaf(mn[i], X, acc[i][t])) : acc[i][t] + P;
+                const float P = (float)(p0[i][t] + p1[i][t]);   // exact below 2^24
+                // sum_k (q_k s + m) x_k = s * 2^(e-14) * sum_k q_k xi_k + m * sum_k x_k
+                acc[i][t] = kInt4 ? fmaf(sc[i] * f, P, fmaf(mn[i], X, acc[i][t])) : fmaf(f, P, acc[i][t]);
               }
             }
           }
@@ -377,14 +414,15 @@ cudaError_t launch_fmt(const TmaGemvArgs& a, int mt, dim3 grid, size_t smem, cud
 
 }  // namespace
 
+size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
+
 size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages) {
   const bool i4 = fmt == FMT_INT4_G32;
-  const int chunk = i4 ? 32 : 16, stride = i4 ? 36 : 20;
-  const int gs = i4 ? klen / 32 : 0;
+  const int nch = klen / (i4 ? 32 : 16);
+  const int cbytes = i4 ? Codes<FMT_INT4_G32>::kStageBytes : Codes<FMT_INT8_ROW>::kStageBytes;
   const int tok_rows = (stage_tokens + mt - 1) / mt * mt;
-  const size_t x_bytes = ((size_t)tok_rows * ((klen / chunk) * stride + gs) * 4 + 127) / 128 * 128;
-  const size_t stage_bytes = (size_t)nm * kTmaConsumers * ((i4 ? klen / 2 : klen) + 4 * gs);
-  return 128 + x_bytes + stage_bytes * stages;
+  const size_t x_bytes = ((size_t)tok_rows * ((size_t)nch * cbytes + 4 * nch + (i4 ? 4 * nch : 0)) + 127) / 128 * 128;
+  return 128 + x_bytes + tma_gemv_stage_bytes(fmt, nm, klen) * stages;
 }
 
 size_t tma_gemv_stage_bytes(int fmt, int nm, int klen) {
@@ -398,6 +436,22 @@ cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, in
   if (a.fmt == FMT_INT4_G32)
     return nm == 2 ? launch_fmt<FMT_INT4_G32, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_INT4_G32, 1>(a, mt, grid, smem, s);
   return nm == 2 ? launch_fmt<FMT_INT8_ROW, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_INT8_ROW, 1>(a, mt, grid, smem, s);
+}
+
+cudaError_t encode_qw_maps(QWMaps* m, int fmt, const QW& w, int N, int K, int ks_len) {
+  const int R = kTmaConsumers;
+  cudaError_t e;
+  if (fmt == FMT_INT4_G32) {
+    e = encode_tmap_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT64, w.q, K / 16, N, K / 2, ks_len / 16, R);
+    if (e != cudaSuccess) return e;
+    e = encode_tmap_2d(&m->scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.scale, K / 32, N, K / 16, ks_len / 32, R);
+    if (e != cudaSuccess) return e;
+    return encode_tmap_2d(&m->mn, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.mn, K / 32, N, K / 16, ks_len / 32, R);
+  }
+  e = encode_tmap_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT64, w.q, K / 8, N, K, ks_len / 8, R);
+  m->scale = m->codes;
+  m->mn = m->codes;
+  return e;
 }
 
 unsigned int tma_gemv_fault_flags(bool clear) {

@@ -1,12 +1,24 @@
 // Launch interface of the TMA-fed GEMV (gemv_tma.cu).
 #pragma once
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace moeffn {
 
 constexpr int kTmaConsumers = 8;  // consumer warps per CTA = rows per stage
 
+// Tensor maps of one K-split matrix: codes (u64 elements), scales, mins (u16).
+struct QWMaps {
+  CUtensorMap codes, scale, mn;
+};
+
 struct TmaGemvArgs {
+  // K-split jobs load [R rows] x [ks_len] boxes through 2-D tensor maps:
+  QWMaps dmap;                 // dense mode (kernel parameter)
+  const QWMaps* maps;          // grouped mode: per expert, device memory
+  const QWMaps* maps_s;        // shared job, device memory
+  int use_maps;                // 1: tensor maps; 0: 1-D bulk copies of whole rows
   int fmt, act;
   QW a0, a1;                   // dense mode: matrices (a1: up, when fused)
   const QW* tab0;              // grouped mode: per-expert tables (device)
@@ -34,6 +46,8 @@ struct TmaGemvArgs {
   int stages;
 };
 
+// Encodes the three maps of W[N][K] for boxes of [rows_per_stage][ks_len].
+cudaError_t encode_qw_maps(QWMaps* m, int fmt, const QW& w, int N, int K, int ks_len);
 size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages);
 size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
 cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, int jobs, cudaStream_t s);

@@ -86,3 +86,17 @@ __device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) 
 }
 
 }  // namespace moeffn
+
+namespace moeffn {
+
+// 2-D tiled TMA load of box {x (inner), y (rows)} of `map` into shared memory,
+// completion counted on `bar`. x * element size must be a multiple of 16.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_addr(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_addr(bar))
+      : "memory");
+}
+
+}  // namespace moeffn

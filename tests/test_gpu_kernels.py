@@ -122,9 +122,10 @@ def test_dense_small(cfg, shape, fmt, M):
     assert_bf16_close(dl.run(inp.x, zero), oracle.layer(inp), "h")
 
 
+@pytest.mark.parametrize("shape", [dict(H=384, I=800), dict(H=256, I=2560)])   # the second splits K (INT8)
 @pytest.mark.parametrize("M", [1, 2, 3, 8])
-def test_shared_expert_small(M):
-    c = synth.scaled_config(3, H=384, I=800)
+def test_shared_expert_small(M, shape):
+    c = synth.scaled_config(3, **shape)
     inp = synth.make_inputs(c, M, 1)
     dl = DeviceLayer(inp)
     assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "h1")
