@@ -340,6 +340,7 @@ def run_ours(args, rank, world, local_rank):
                 "d2h_bytes_per_step": int(inp.residual.nbytes),
             },
             "gpu_launches": int(launches),
+            "device_faults": lib.device_faults(True),
             "clocks": clocks,
         }
     if dist is not None:

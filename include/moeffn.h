@@ -171,6 +171,14 @@ size_t moe_workspace_bytes(const moeffn_moe_plan* plan, int M);
 int moe_layer(moeffn_moe_plan* plan, const uint16_t* x, uint16_t* residual, int M, int32_t* topk_idx_out,
               void* ws, size_t ws_bytes, moeffn_stream_t stream);
 
+/* Failure detection. Pipeline waits inside the kernels are bounded (about one
+ * second); a wait that runs out sets a bit in a device fault word and the
+ * kernel finishes without its result instead of hanging. Returns the word
+ * (bit 0: a pipeline barrier wait timed out; bit 1: a launch with an invalid
+ * pipeline depth was refused) and clears it if `clear` != 0.
+ * Synchronous (a device-to-host copy); not for the hot path. */
+unsigned int moeffn_device_faults(int clear);
+
 /* ---- Per-launch timing (tracing) ------------------------------------------
  * No counterpart on the pages (they time host phases with PhaseCounters).
  * Off by default. While enabled, every kernel launch of the library is

@@ -74,6 +74,7 @@ _SIGS = {
     "moe_layer": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _sz, _vp]),
     "moeffn_test_dequant": (_i, [ctypes.POINTER(_QWeight), _vp, _vp, _vp]),
     "moeffn_profile_enable": (_i, [_i]),
+    "moeffn_device_faults": (ctypes.c_uint, [_i]),
     "moeffn_profile_read": (_i, [ctypes.c_char_p, _i, _vp, _vp, _i, ctypes.POINTER(_i)]),
     "moeffn_test_topk_from_logits": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
@@ -266,6 +267,11 @@ def moe_layer(plan: MoePlan, x: torch.Tensor, residual: torch.Tensor, topk_idx_o
     return residual
 
 
+def device_faults(clear: bool = True) -> int:
+    """Fault word of the kernels' bounded waits (0: none); blocking."""
+    return int(_lib.moeffn_device_faults(1 if clear else 0))
+
+
 def profile_enable(on: bool = True) -> None:
     """Bracket each library kernel launch with CUDA events (see moeffn_profile_read)."""
     _check(_lib.moeffn_profile_enable(1 if on else 0))
@@ -310,4 +316,4 @@ def test_topk_from_logits(logits: torch.Tensor, top_k: int, stream=None):
 
 __all__ = ["ffn_dense", "ffn_shared_expert", "moe_router_topk", "moe_layer", "MoePlan", "QWeight", "FFN",
            "qweight_from_arrays", "upload_qweight", "upload_ffn", "plain_weight", "workspace_bytes", "alloc_workspace", "test_dequant",
-           "test_topk_from_logits", "profile_enable", "profile_read", "MoeffnError", "LIB_PATH"]
+           "test_topk_from_logits", "profile_enable", "profile_read", "device_faults", "MoeffnError", "LIB_PATH"]

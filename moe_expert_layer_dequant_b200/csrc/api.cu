@@ -136,9 +136,11 @@ TmaGeom tma_geom(int fmt, int nm, int klen, int want_tokens) {
   g.tokens = std::max(1, std::min(want_tokens, t));
   const size_t base = tma_gemv_smem(fmt, nm, klen, g.tokens, g.mt, 0);
   const size_t st = tma_gemv_stage_bytes(fmt, nm, klen);
-  const int stages = base + 2 * st <= kTmaSmemBudget ? (int)std::min<size_t>(6, (kTmaSmemBudget - base) / st) : 0;
+  int stages = base + 2 * st <= kTmaSmemBudget ? (int)std::min<size_t>(8, (kTmaSmemBudget - base) / st) : 0;
+  // Each ring slot must belong to one consumer group (see gemv_tma.cu).
+  stages -= stages % kTmaGroups;
   g.stages = stages;
-  g.ok = stages >= 2;
+  g.ok = stages >= kTmaGroups && stages >= 2;
   return g;
 }
 
@@ -364,6 +366,11 @@ struct moeffn_moe_plan {
 extern "C" {
 
 const char* moeffn_last_error(void) { return g_last_error.c_str(); }
+
+unsigned int moeffn_device_faults(int clear) {
+  // Blocking read of the kernels' fault words (bounded waits that ran out).
+  return tma_gemv_fault_flags(clear != 0);
+}
 
 size_t moeffn_workspace_bytes(int kind, int M, int H, int I, int E, int top_k) {
   if (M < 1 || H < 1) return 0;

@@ -151,3 +151,14 @@ __device__ __forceinline__ void int8_word_dequant(uint32_t w, float s, float (&o
 }
 
 }  // namespace moeffn
+
+namespace moeffn {
+
+// Programmatic dependent launch: a kernel launched with the PDL attribute may
+// start while its predecessor in the stream still runs. It must call
+// pdl_wait() before touching memory the predecessor writes or reads; weights
+// (never written by kernels) may be streamed before that.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace moeffn

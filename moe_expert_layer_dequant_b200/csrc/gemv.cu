@@ -15,6 +15,7 @@
 //                  slot order;
 //  * shared job  : the MoE layer's shared expert, over all M tokens.
 #include "gemv.cuh"
+#include "launch.cuh"
 
 namespace moeffn {
 
@@ -215,6 +216,8 @@ __device__ __forceinline__ Job gateup_job(const GateUpArgs& a) {
 template <int FMT, int MT>
 __global__ void __launch_bounds__(kThreads, 2) k_gateup(const GateUpArgs a) {
   extern __shared__ __align__(16) float smem[];
+  pdl_launch_dependents();
+  pdl_wait();
   const Job job = gateup_job(a);
   if (!job.valid) return;
   const int row0 = blockIdx.x * a.rows_per_cta;
@@ -281,6 +284,8 @@ __device__ __forceinline__ Job down_job(const DownArgs& a) {
 template <int FMT, int MT>
 __global__ void __launch_bounds__(kThreads, 2) k_down(const DownArgs a) {
   extern __shared__ __align__(16) float smem[];
+  pdl_launch_dependents();
+  pdl_wait();
   const Job job = down_job(a);
   if (!job.valid || job.ntok == 0) return;
   const bool shared_job = (a.offsets != nullptr && blockIdx.z >= a.routed_jobs);
@@ -336,8 +341,7 @@ cudaError_t launch(KernelT kern, dim3 grid, size_t smem, cudaStream_t s, const A
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kThreads), smem, s, a);
 }
 
 }  // namespace

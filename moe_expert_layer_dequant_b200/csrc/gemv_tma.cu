@@ -21,6 +21,7 @@
 #include "gemv_tma.cuh"
 #include "sync.cuh"
 #include "tmap.cuh"
+#include "launch.cuh"
 
 namespace moeffn {
 
@@ -123,13 +124,25 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-template <int FMT, int MT, int NM, int NC>
-__global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_constant__ TmaGemvArgs a) {
+// NC consumer warps per group, G groups: group g takes the stages s with
+// s % G == g, one row of the stage per warp (R = NC rows per stage). The ring
+// depth S is a multiple of G, so every slot is waited on by one group only,
+// in stage order: a waiter is never two phases ahead of a slot's barriers
+// (whose phase parity would then alias the previous use).
+template <int FMT, int MT, int NM, int NC, int G>
+__global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_constant__ TmaGemvArgs a) {
   using C = Codes<FMT>;
   constexpr bool kInt4 = (FMT == FMT_INT4_G32);
-  constexpr int R = NC;  // rows per stage: one per consumer warp
+  constexpr int R = NC;  // rows per stage
   extern __shared__ __align__(128) uint8_t smem[];
 
+  // No global memory access (weights included) before the previous kernel in
+  // the stream has completed: only the launch itself overlaps it.
+  pdl_wait();
+  if (a.stages % G != 0 || a.stages > 8) {   // ring depth the host must not choose
+    if (threadIdx.x == 0) atomicOr(&g_fault_flags, 2u);
+    return;
+  }
   const Job job = decode_job(a);
   if (!job.valid || job.ntok == 0) return;
   const int k0 = blockIdx.y * a.ks_len;
@@ -181,7 +194,10 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
   const int row_bytes = kInt4 ? job.K / 2 : job.K;
   const int row_groups = job.K / 32;
 
-  if (warp == NC) {
+  // The next kernel in the stream may be scheduled now; it waits for this
+  // grid's completion before reading what this grid writes.
+  pdl_launch_dependents();
+  if (warp == NC * G) {
     // ---------------- producer ----------------
     if (lane == 0) {
       for (int s = 0; s < total; ++s) {
@@ -224,12 +240,12 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
   }
 
   // ---------------- consumers ----------------
-  const int nthreads = NC * 32;
+  const int nthreads = NC * G * 32;
+  const int grp = warp / NC, wr = warp - grp * NC;  // group, row of the stage
   const uint16_t* src = job.shared ? a.x_s : a.x;
   const int ld = job.shared ? job.K : a.ld_x;
-  int s = 0;
   bool dead = false;
-  for (int tb = 0; tb < job.ntok; tb += a.stage_tokens) {
+  for (int tb = 0, tbi = 0; tb < job.ntok; tb += a.stage_tokens, ++tbi) {
     const int tn = min(a.stage_tokens, job.ntok - tb);
     consumer_sync(nthreads);
     // Stage token rows tb..tb+tn (K slice) chunk by chunk: int16 fixed point,
@@ -266,22 +282,22 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
         frexpf(amax, &e);
         e -= 1;                                   // amax in [2^e, 2^(e+1))
       }
-      int16_t* dst = reinterpret_cast<int16_t*>(xi + (size_t)r * tok_stride + c * C::kStageBytes);
+      int16_t* dst = reinterpret_cast<int16_t*>(xi + r * tok_stride + c * C::kStageBytes);
+      constexpr int kW = (C::kChunk == 32 ? 8 : 4);   // codes per 32-bit word
 #pragma unroll
       for (int j = 0; j < C::kChunk; ++j) {
         const float f = bf16_bits_to_float(v[j]);
-        const int word = j / (C::kChunk == 32 ? 8 : 4), pos = j % (C::kChunk == 32 ? 8 : 4);
-        dst[word * (C::kChunk == 32 ? 8 : 4) + C::slot_of(pos)] =
-            (int16_t)(amax > 0.f ? __float2int_rn(ldexpf(f, 14 - e)) : 0);
+        dst[(j / kW) * kW + C::slot_of(j % kW)] = (int16_t)(amax > 0.f ? __float2int_rn(ldexpf(f, 14 - e)) : 0);
       }
       xf[r * nch + c] = amax > 0.f ? ldexpf(1.0f, e - 14) : 0.f;
       if (kInt4) xsum[r * nch + c] = sum;
     }
     consumer_sync(nthreads);
 
-    for (int rs = 0; rs < row_stages; ++rs, ++s) {
+    for (int rs = grp; rs < row_stages; rs += G) {
+      const int s = tbi * row_stages + rs;
       const int slot = s % S, use = s / S;
-      const int n = r0 + rs * R + warp;
+      const int n = r0 + rs * R + wr;
       float row_scale[NM];
       if (!kInt4 && n < r1) {
 #pragma unroll
@@ -291,38 +307,35 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
       // computing but still takes part in every barrier below.
       if (!dead && !mbar_wait(&full[slot], use & 1)) dead = true;
       if (!dead && n < r1) {
-        const uint8_t* st = stage0 + (size_t)slot * stage_bytes;
-        const uint8_t* codes[NM];
-        const __half* scl[NM];
-        const __half* mns[NM];
+        // 32-bit byte offsets from the stage start (shared memory).
+        const uint8_t* st = stage0 + slot * (int)stage_bytes;
+        int o_code[NM], o_sc[NM];
 #pragma unroll
         for (int i = 0; i < NM; ++i) {
-          codes[i] = st + ((size_t)i * R + warp) * cs + lane * 16;
-          scl[i] = reinterpret_cast<const __half*>(st + (size_t)NM * R * cs) + ((size_t)i * R + warp) * gst + lane;
-          mns[i] = reinterpret_cast<const __half*>(st + (size_t)NM * R * cs + (size_t)NM * R * gst * 2) +
-                   ((size_t)i * R + warp) * gst + lane;
+          o_code[i] = (i * R + wr) * cs + lane * 16;
+          o_sc[i] = NM * R * cs + ((i * R + wr) * gst + lane) * 2;
         }
+        const int mn_off = NM * R * gst * 2;   // mins follow the scales
         for (int tc = 0; tc < tn; tc += MT) {
           float acc[NM][MT];
 #pragma unroll
           for (int i = 0; i < NM; ++i)
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[i][t] = 0.f;
-          const uint8_t* xl = xi + (size_t)tc * tok_stride + lane * C::kStageBytes;
-          const int iters = (nch - lane + 31) >> 5;
-          for (int it = 0; it < iters; ++it) {
-            const int c = lane + 32 * it;
+          int ox = tc * tok_stride + lane * C::kStageBytes;   // staged activations
+          int of = tc * nch + lane;                            // factors / sums
+          int oc = 0, og = 0;                                  // code / scale advance
+          for (int c = lane; c < nch; c += 32, ox += 32 * C::kStageBytes, of += 32, oc += 512, og += 64) {
             uint4 wv[NM];
             float sc[NM], mn[NM];
 #pragma unroll
             for (int i = 0; i < NM; ++i) {
-              wv[i] = *reinterpret_cast<const uint4*>(codes[i] + it * 512);
+              wv[i] = *reinterpret_cast<const uint4*>(st + o_code[i] + oc);
               if (kInt4) {
-                sc[i] = __half2float(scl[i][it * 32]);
-                mn[i] = __half2float(mns[i][it * 32]);
+                sc[i] = __half2float(*reinterpret_cast<const __half*>(st + o_sc[i] + og));
+                mn[i] = __half2float(*reinterpret_cast<const __half*>(st + o_sc[i] + og + mn_off));
               }
             }
-            const uint8_t* xc = xl + it * 32 * C::kStageBytes;
             int p0[NM][MT], p1[NM][MT];
 #pragma unroll
             for (int i = 0; i < NM; ++i)
@@ -333,7 +346,7 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
               for (int q = 0; q < 4; ++q) {
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                  const uint4 x4 = *reinterpret_cast<const uint4*>(xc + (size_t)t * tok_stride + q * 16);
+                  const uint4 x4 = *reinterpret_cast<const uint4*>(xi + ox + t * tok_stride + q * 16);
 #pragma unroll
                   for (int i = 0; i < NM; ++i) {
                     const uint32_t w = q == 0 ? wv[i].x : q == 1 ? wv[i].y : q == 2 ? wv[i].z : wv[i].w;
@@ -346,7 +359,7 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
               for (int h = 0; h < 2; ++h) {
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                  const uint4 x4 = *reinterpret_cast<const uint4*>(xc + (size_t)t * tok_stride + h * 16);
+                  const uint4 x4 = *reinterpret_cast<const uint4*>(xi + ox + t * tok_stride + h * 16);
 #pragma unroll
                   for (int i = 0; i < NM; ++i) {
                     const uint32_t w0 = h == 0 ? wv[i].x : wv[i].z, w1 = h == 0 ? wv[i].y : wv[i].w;
@@ -357,8 +370,8 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
             }
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-              const float f = xf[(tc + t) * nch + c];
-              const float X = kInt4 ? xsum[(tc + t) * nch + c] : 0.f;
+              const float f = xf[of + t * nch];
+              const float X = kInt4 ? xsum[of + t * nch] : 0.f;
 #pragma unroll
               for (int i = 0; i < NM; ++i) {
                 const float P = (float)(p0[i][t] + p1[i][t]);   // exact below 2^24
@@ -397,19 +410,21 @@ __global__ void __launch_bounds__(32 * (NC + 1), 1) k_gemv_tma(const __grid_cons
   }
 }
 
-template <int FMT, int MT, int NM, int NC>
+template <int FMT, int MT, int NM>
 cudaError_t launch_one(const TmaGemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-  auto kern = k_gemv_tma<FMT, MT, NM, NC>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  kern<<<grid, 32 * (NC + 1), smem, s>>>(a);
-  return cudaGetLastError();
+  auto kern = k_gemv_tma<FMT, MT, NM, kTmaConsumers, kTmaGroups>;
+  static size_t smem_set = 0;  // largest dynamic shared memory opted in so far
+  if (smem > smem_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    if (e != cudaSuccess) return e;
+    smem_set = 227 * 1024;
+  }
+  return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * kTmaGroups + 1)), smem, s, a);
 }
 
 template <int FMT, int NM>
 cudaError_t launch_fmt(const TmaGemvArgs& a, int mt, dim3 grid, size_t smem, cudaStream_t s) {
-  return mt == 1 ? launch_one<FMT, 1, NM, kTmaConsumers>(a, grid, smem, s)
-                 : launch_one<FMT, 2, NM, kTmaConsumers>(a, grid, smem, s);
+  return mt == 1 ? launch_one<FMT, 1, NM>(a, grid, smem, s) : launch_one<FMT, 2, NM>(a, grid, smem, s);
 }
 
 }  // namespace

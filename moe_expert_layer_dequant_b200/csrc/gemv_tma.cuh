@@ -6,7 +6,8 @@
 
 namespace moeffn {
 
-constexpr int kTmaConsumers = 8;  // consumer warps per CTA = rows per stage
+constexpr int kTmaConsumers = 8;  // consumer warps per group = rows per stage
+constexpr int kTmaGroups = 2;     // consumer groups, taking alternate stages
 
 // Tensor maps of one K-split matrix: codes (u64 elements), scales, mins (u16).
 struct QWMaps {

@@ -8,28 +8,31 @@
 // fp16 routing weights. Here none of it leaves the GPU: one kernel computes the
 // logits (plus the shared-expert gate logit), a single-CTA kernel selects the
 // top-k, computes the weights and builds the grouped permutation.
+#include <algorithm>
+
+#include "launch.cuh"
 #include "route.cuh"
 
 namespace moeffn {
 
 namespace {
 
-constexpr int kRouterWarps = 8;
+constexpr int kRouterThreads = 128;
 
-// logits[t][e] = Wr[e] . x[t] (fp32 accumulate); row e == E is the shared
-// expert gate vector (bf16), written to gate_logit[t].
-__global__ void __launch_bounds__(kRouterWarps * 32) k_router_logits(const RouterArgs a) {
+// logits[t][e] = Wr[e] . x[t] (fp32 accumulate), one CTA per (token, row);
+// row e == E is the shared expert gate vector (bf16), written to gate_logit[t].
+__global__ void __launch_bounds__(kRouterThreads) k_router_logits(const RouterArgs a) {
+  __shared__ float red[kRouterThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
   const int t = blockIdx.x;
-  const int e = blockIdx.y * kRouterWarps + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  const int rows = a.E + (a.w_sg != nullptr ? 1 : 0);
-  if (e >= rows) return;
+  const int e = blockIdx.y;
+  const bool gate_row = (e == a.E);
   const uint16_t* x = a.x + (size_t)t * a.H;
   float acc = 0.f;
-  const bool gate_row = (e == a.E);
   if (!gate_row && a.router_f32) {
     const float* w = reinterpret_cast<const float*>(a.router) + (size_t)e * a.H;
-    for (int k = lane * 4; k < a.H; k += 128) {
+    for (int k = threadIdx.x * 4; k < a.H; k += kRouterThreads * 4) {
       const float4 wv = *reinterpret_cast<const float4*>(w + k);
       const uint2 xv = *reinterpret_cast<const uint2*>(x + k);
       acc = fmaf(wv.x, __uint_as_float(xv.x << 16), acc);
@@ -39,7 +42,7 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_logits(const Route
     }
   } else {
     const uint16_t* w = gate_row ? a.w_sg : reinterpret_cast<const uint16_t*>(a.router) + (size_t)e * a.H;
-    for (int k = lane * 8; k < a.H; k += 256) {
+    for (int k = threadIdx.x * 8; k < a.H; k += kRouterThreads * 8) {
       const uint4 wv = *reinterpret_cast<const uint4*>(w + k);
       const uint4 xv = *reinterpret_cast<const uint4*>(x + k);
       const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -51,44 +54,77 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_logits(const Route
     }
   }
   acc = warp_sum(acc);
-  if (lane == 0) {
-    if (gate_row) a.gate_logit[t] = acc;
-    else a.logits[(size_t)t * a.E + e] = acc;
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+    for (int i = 0; i < kRouterThreads / 32; ++i) v += red[i];   // fixed order
+    if (gate_row) a.gate_logit[t] = v;
+    else a.logits[(size_t)t * a.E + e] = v;
   }
 }
 
-// One CTA: per token the k largest logits ordered by (logit desc, index asc),
-// softmax over them times the per-expert scale (ones), rounded to fp16; then
-// the stable expert-grouped order of the pairs p = t*k + r.
+// (value, index) order of the top-k: larger value first, lower index on ties.
+__device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+// One CTA. Each warp selects the top-k of its tokens: every lane holds E/32
+// logits; k rounds of a warp-wide arg-max, the winner's lane retires it.
+// Weights: softmax over the k selected logits times the per-expert scale
+// (ones), rounded to fp16. Then the stable expert-grouped order of the pairs
+// p = t*k + r (counts, offsets, union, placement by warp 0).
 __global__ void __launch_bounds__(1024) k_route(const RouteArgs a) {
   extern __shared__ int sm[];
+  pdl_launch_dependents();
+  pdl_wait();
   int* counts = sm;                 // [E]
   int* running = sm + a.E;          // [E]
   int* offs = sm + 2 * a.E;         // [E+1]
   const int P = a.M * a.k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  const int per_lane = (a.E + 31) / 32;
 
-  for (int t = threadIdx.x; t < a.M; t += blockDim.x) {
+  for (int t = warp; t < a.M; t += nwarps) {
     const float* l = a.logits + (size_t)t * a.E;
-    int chosen[kMaxTopK];
-    float val[kMaxTopK];
-    for (int r = 0; r < a.k; ++r) {
-      int best = -1;
-      float bv = 0.f;
-      for (int e = 0; e < a.E; ++e) {
-        bool taken = false;
-        for (int q = 0; q < r; ++q) taken |= (chosen[q] == e);
-        if (taken) continue;
-        const float v = l[e];
-        if (best < 0 || v > bv) { best = e; bv = v; }   // strict '>' keeps the lower index on ties
-      }
-      chosen[r] = best;
-      val[r] = bv;
+    float lv[kMaxExperts / 32];
+    unsigned taken = 0;
+#pragma unroll
+    for (int j = 0; j < kMaxExperts / 32; ++j) {
+      const int e = lane + 32 * j;
+      lv[j] = (j < per_lane && e < a.E) ? l[e] : 0.f;
     }
-    float z[kMaxTopK], s = 0.f;
-    for (int r = 0; r < a.k; ++r) { z[r] = expf(val[r] - val[0]); s += z[r]; }
+    float top0 = 0.f, zsum = 0.f;
+    float zr[kMaxTopK];
+    int ir[kMaxTopK];
     for (int r = 0; r < a.k; ++r) {
-      a.idx[t * a.k + r] = chosen[r];
-      a.w[t * a.k + r] = __half2float(__float2half_rn(z[r] / s));
+      float bv = -INFINITY;   // lanes without a candidate never win
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int j = 0; j < kMaxExperts / 32; ++j) {
+        const int e = lane + 32 * j;
+        if (j < per_lane && e < a.E && !((taken >> j) & 1u) && beats(lv[j], e, bv, bi)) {
+          bv = lv[j];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (beats(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (r == 0) top0 = bv;
+      zr[r] = expf(bv - top0);
+      ir[r] = bi;
+      zsum += zr[r];
+    }
+    if (lane == 0) {
+      for (int r = 0; r < a.k; ++r) {
+        a.idx[t * a.k + r] = ir[r];
+        a.w[t * a.k + r] = __half2float(__float2half_rn(zr[r] / zsum));
+      }
     }
   }
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
@@ -111,7 +147,6 @@ __global__ void __launch_bounds__(1024) k_route(const RouteArgs a) {
   // Stable placement: warp 0 walks the pairs in order, 32 at a time; equal
   // experts inside a chunk are ranked by lane (match_any + popc).
   if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
     for (int base = 0; base < P; base += 32) {
       const int p = base + lane;
       const bool act = p < P;
@@ -135,16 +170,13 @@ __global__ void __launch_bounds__(1024) k_route(const RouteArgs a) {
 
 cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t s) {
   const int rows = a.E + (a.w_sg != nullptr ? 1 : 0);
-  const dim3 grid(a.M, (rows + kRouterWarps - 1) / kRouterWarps);
-  k_router_logits<<<grid, kRouterWarps * 32, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(k_router_logits, dim3(a.M, rows), dim3(kRouterThreads), 0, s, a);
 }
 
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)(3 * a.E + 1) * sizeof(int);
-  const int threads = a.M >= 1024 ? 1024 : ((a.M + 31) / 32) * 32 < 128 ? 128 : ((a.M + 31) / 32) * 32;
-  k_route<<<1, threads, smem, s>>>(a);
-  return cudaGetLastError();
+  const int threads = std::min(1024, std::max(128, a.M * 32));   // a warp per token
+  return launch_pdl(k_route, dim3(1), dim3(threads), smem, s, a);
 }
 
 }  // namespace moeffn

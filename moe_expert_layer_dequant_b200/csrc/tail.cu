@@ -14,6 +14,7 @@
 //               seeded with the gated shared expert; no norm in the tail).
 //               seed = bf16(bf16(s) * sigmoid(gate_logit)) with s the shared
 //               expert's down output, or 0 without a shared expert.
+#include "launch.cuh"
 #include "tail.cuh"
 
 namespace moeffn {
@@ -27,6 +28,8 @@ __device__ __forceinline__ float sum_splits(const float* d, int splits, size_t s
 }
 
 __global__ void k_tail_elementwise(const TailArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
   const size_t total = (size_t)a.M * a.N;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
     const int t = (int)(i / a.N), n = (int)(i - (size_t)t * a.N);
@@ -53,6 +56,8 @@ __global__ void k_tail_elementwise(const TailArgs a) {
 
 __global__ void __launch_bounds__(512) k_tail_rmsnorm(const TailArgs a) {
   extern __shared__ float red[];
+  pdl_launch_dependents();
+  pdl_wait();
   const int t = blockIdx.x;
   float ss = 0.f;
   for (int n = threadIdx.x; n < a.N; n += blockDim.x) {
@@ -80,12 +85,12 @@ __global__ void __launch_bounds__(512) k_tail_rmsnorm(const TailArgs a) {
 
 cudaError_t launch_tail(const TailArgs& a, cudaStream_t s) {
   if (a.mode == TAIL_RMSNORM) {
-    k_tail_rmsnorm<<<a.M, 512, 16 * sizeof(float), s>>>(a);
+    return launch_pdl(k_tail_rmsnorm, dim3(a.M), dim3(512), 16 * sizeof(float), s, a);
   } else {
     const size_t total = (size_t)a.M * a.N;
     int blocks = (int)((total + 255) / 256);
     if (blocks > 148 * 8) blocks = 148 * 8;
-    k_tail_elementwise<<<blocks, 256, 0, s>>>(a);
+    return launch_pdl(k_tail_elementwise, dim3(blocks), dim3(256), 0, s, a);
   }
   return cudaGetLastError();
 }
