@@ -117,6 +117,24 @@ const char* moeffn_last_error(void);
 int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act,
               void* ws, size_t ws_bytes, moeffn_stream_t stream);
 
+/* Dense FFN plus residual add without a caller workspace. No counterpart on
+ * the pages. For callers that cannot allocate device memory at the point of
+ * the call: code inside a stream capture that must not add allocations,
+ * runtimes that budget all device memory before they start, plugins handed
+ * only input and output pointers. Computes exactly what ffn_dense computes,
+ * with its scratch in a fixed array inside the library that is
+ * MOEFFN_NOALLOC_SCRATCH_BYTES long and stays allocated on every GPU that
+ * loads the library until the process exits. Allocates nothing. A call whose
+ * scratch need (moeffn_workspace_bytes of MOEFFN_KIND_DENSE) is larger than
+ * the array returns MOEFFN_ERR_WORKSPACE before any launch. The first call on
+ * a device looks up the array's device address there (with that device
+ * current); make that first call before any stream capture. Every call uses
+ * the same array: calls that can overlap on the GPU (other streams, other
+ * host threads) race on it and must be serialized by the caller. */
+#define MOEFFN_NOALLOC_SCRATCH_BYTES (4u << 20)
+int ffn_dense_noalloc(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act,
+                      moeffn_stream_t stream);
+
 /* Gemma shared-expert branch with its trailing post-FFN RMSNorm:
  *   h1[t] = bf16(h / sqrt(mean(h^2) + eps) * norm_w), h = bf16(FFN(x_t))
  * turbospark-runtime 0.1.0, src/families/gemma4/shared_expert.rs,

@@ -66,6 +66,7 @@ _SIGS = {
     "moeffn_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "moeffn_last_error": (ctypes.c_char_p, []),
     "ffn_dense": (_i, [ctypes.POINTER(_FFN), _vp, _vp, _i, _i, _vp, _sz, _vp]),
+    "ffn_dense_noalloc": (_i, [ctypes.POINTER(_FFN), _vp, _vp, _i, _i, _vp]),
     "ffn_shared_expert": (_i, [ctypes.POINTER(_FFN), _vp, _vp, _f, _vp, _i, _i, _vp, _sz, _vp]),
     "moe_router_topk": (_i, [ctypes.POINTER(_QWeight), _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_plan_create": (_i, [ctypes.POINTER(_MoeDesc), ctypes.POINTER(_vp)]),
@@ -199,6 +200,23 @@ def ffn_dense(w: FFN, x: torch.Tensor, residual: torch.Tensor, act: str = "silu"
     return residual
 
 
+NOALLOC_SCRATCH_BYTES = 4 << 20
+
+
+def ffn_dense_noalloc(w: FFN, x: torch.Tensor, residual: torch.Tensor, act: str = "silu", stream=None) -> torch.Tensor:
+    """ffn_dense with the library's fixed scratch array instead of a workspace.
+
+    For callers that cannot allocate device memory when they call; the call
+    allocates nothing. Raises MoeffnError (status -3) when the call needs more
+    than NOALLOC_SCRATCH_BYTES of scratch. All calls share one array, so calls
+    that may overlap on the GPU must be serialized by the caller.
+    """
+    M = x.shape[0]
+    f = w.c()
+    _check(_lib.ffn_dense_noalloc(ctypes.byref(f), _ptr(x), _ptr(residual), M, ACTS[act], _stream(stream)))
+    return residual
+
+
 def ffn_shared_expert(w: FFN, x: torch.Tensor, norm_w: torch.Tensor, h1_out: torch.Tensor, act: str = "gelu_tanh",
                       eps: float = 1e-6, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """h1_out <- RMSNorm(bf16(FFN(x))) * norm_w; all bf16."""
@@ -314,6 +332,6 @@ def test_topk_from_logits(logits: torch.Tensor, top_k: int, stream=None):
     return idx, w, perm, offs, uni[: int(nu.item())]
 
 
-__all__ = ["ffn_dense", "ffn_shared_expert", "moe_router_topk", "moe_layer", "MoePlan", "QWeight", "FFN",
+__all__ = ["ffn_dense", "ffn_dense_noalloc", "ffn_shared_expert", "moe_router_topk", "moe_layer", "MoePlan", "QWeight", "FFN",
            "qweight_from_arrays", "upload_qweight", "upload_ffn", "plain_weight", "workspace_bytes", "alloc_workspace", "test_dequant",
            "test_topk_from_logits", "profile_enable", "profile_read", "device_faults", "MoeffnError", "LIB_PATH"]
