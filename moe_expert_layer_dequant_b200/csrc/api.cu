@@ -9,6 +9,7 @@
 #include "../../include/moeffn.h"
 #include "common.cuh"
 #include "gemv.cuh"
+#include "gemm_tc.cuh"
 #include "gemv_tma.cuh"
 #include "tmap.cuh"
 #include "prof.cuh"
@@ -152,6 +153,35 @@ int stage_tokens(int fmt, int klen, int want) {
 
 int mt_for(int tokens) { return tokens <= 1 ? 1 : 2; }
 
+// ---- tensor-core GEMM eligibility and geometry ------------------------------
+
+constexpr int kTcMinTokens = 3;      // dense: token rows from which the GEMM replaces the GEMV
+constexpr int kTcMinMoeTokens = 8;   // MoE layer: token rows from which the grouped GEMMs are used
+
+bool tc_ok(const moeffn_qweight& w) {
+  if (!aligned16(w.q)) return false;
+  if (w.format == MOEFFN_Q_INT4_AFFINE_G32) return w.cols % 256 == 0 && aligned16(w.scale) && aligned16(w.min);
+  return w.format == MOEFFN_Q_INT8_ROW && w.cols % 128 == 0;
+}
+bool tc_ok(const moeffn_ffn& f) { return tc_ok(f.gate) && tc_ok(f.up) && tc_ok(f.down); }
+
+// Token tile (MMA N) for an expected number of token rows per weight matrix.
+int tc_nt(int tokens) {
+  int nt = 16;
+  while (nt < tokens && nt < 256) nt *= 2;
+  return nt;
+}
+
+// K split of a down-projection GEMM: about `want` splits, at most `max_splits`,
+// slices a multiple of the weight stage K.
+int tc_down_slice(int K, int fmt, int want, int max_splits) {
+  const int kt = tc_k_tile(fmt);
+  const int s = std::max(1, std::min(want, max_splits));
+  int ks = ((K + s - 1) / s + kt - 1) / kt * kt;
+  while ((K + ks - 1) / ks > max_splits) ks += kt;
+  return ks;
+}
+
 // ---- workspace layout ------------------------------------------------------
 
 struct Carve {
@@ -191,6 +221,7 @@ struct MoeWS {
   uint16_t* acts_s;
   float* d;
   float* d_s;
+  uint16_t* xg;      // token rows in pair-slot order (grouped GEMM operand)
 };
 
 // Down-projection K split shared by the routed and the shared expert jobs.
@@ -223,6 +254,7 @@ MoeWS carve_moe(Carve& c, int M, int H, int Ie, int Is, int E, int k) {
   w.acts_s = c.take<uint16_t>((size_t)M * std::max(Is, 0));
   w.d = c.take<float>((size_t)sp.routed * P * H);
   w.d_s = c.take<float>((size_t)sp.shared * M * H);
+  w.xg = c.take<uint16_t>(P * H);
   return w;
 }
 
@@ -250,10 +282,60 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 // ---- shared FFN launch (dense mode) ---------------------------------------
 
+// Gate/up + activation and the down projection (fp32 K-split partials in
+// w.d); returns the number of splits written through *splits_out.
 int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, int act, const DenseWS& w,
-                  cudaStream_t s) {
+                  cudaStream_t s, int* splits_out) {
   const int fmt = f.gate.format;
+  if (M >= kTcMinTokens && tc_ok(f) && aligned16(x)) {
+    const int nt = tc_nt(M), tt = (M + nt - 1) / nt;
+    TcGemmArgs g{};
+    g.fmt = fmt;
+    g.act = act;
+    g.mode = TC_GATEUP;
+    g.nt = nt;
+    g.N = I;
+    g.K = H;
+    g.M = M;
+    g.slots = M;
+    g.out_act = w.acts;
+    g.ks_len = H;
+    g.token_tiles = tt;
+    g.rscale0 = static_cast<const __half*>(f.gate.scale);
+    g.rscale1 = static_cast<const __half*>(f.up.scale);
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, x, M, H, nt), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w0, fmt, to_qw(f.gate), I, H, 64), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w1, fmt, to_qw(f.up), I, H, 64), "tensor map encode");
+    {
+      ProfScope ps("gateup_gemm_tc", s);
+      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (I + 63) / 64, 1, 1, s), "gate/up GEMM launch");
+    }
+    TcGemmArgs d{};
+    d.fmt = fmt;
+    d.mode = TC_DOWN;
+    d.nt = nt;
+    d.N = H;
+    d.K = I;
+    d.M = M;
+    d.slots = M;
+    d.out_d = w.d;
+    d.token_tiles = tt;
+    d.rscale0 = static_cast<const __half*>(f.down.scale);
+    const int row_tiles = (H + 127) / 128;
+    const int want = (kSMs + row_tiles * tt - 1) / (row_tiles * tt);
+    d.ks_len = tc_down_slice(I, fmt, want, down_splits_any(I));
+    const int splits = (I + d.ks_len - 1) / d.ks_len;
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, M, I, nt), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&d.w0, fmt, to_qw(f.down), H, I, 128), "tensor map encode");
+    {
+      ProfScope ps("down_gemm_tc", s);
+      MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, splits, 1, s), "down GEMM launch");
+    }
+    *splits_out = splits;
+    return MOEFFN_OK;
+  }
   const int ks = down_slice(I, fmt), splits = down_splits(I, fmt);
+  *splits_out = splits;
   const TmaGeom gu = tma_geom(fmt, 2, H, M);
   const TmaGeom dn = tma_geom(fmt, 1, ks, M);
   if (tma_ok(f) && gu.ok && dn.ok) {
@@ -361,6 +443,11 @@ struct moeffn_moe_plan {
   QW* d_down = nullptr;
   QWMaps* d_maps = nullptr;    // [E] tensor maps of the expert down matrices (K split)
   QWMaps* d_maps_s = nullptr;  // [1] shared expert down (K split)
+  bool tc = false;             // tensor-core GEMM maps built
+  TcMaps* d_tc_gate = nullptr; // [E] (64-row boxes)
+  TcMaps* d_tc_up = nullptr;   // [E] (64-row boxes)
+  TcMaps* d_tc_down = nullptr; // [E] (128-row boxes)
+  TcMaps tc_sg{}, tc_su{}, tc_sd{};
 };
 
 extern "C" {
@@ -413,13 +500,14 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
   Carve cw{static_cast<char*>(ws)};
   const DenseWS d = carve_dense(cw, M, H, I);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s)) != MOEFFN_OK) return rc;
+  int splits = 0;
+  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits)) != MOEFFN_OK) return rc;
   TailArgs t{};
   t.mode = TAIL_RESIDUAL;
   t.M = M;
   t.N = H;
   t.d = d.d;
-  t.splits = down_splits(I, w->gate.format);
+  t.splits = splits;
   t.slots = M;
   t.res = residual;
   {
@@ -451,13 +539,14 @@ int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* no
   Carve cw{static_cast<char*>(ws)};
   const DenseWS d = carve_dense(cw, M, H, I);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s)) != MOEFFN_OK) return rc;
+  int splits = 0;
+  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits)) != MOEFFN_OK) return rc;
   TailArgs t{};
   t.mode = TAIL_RMSNORM;
   t.M = M;
   t.N = H;
   t.d = d.d;
-  t.splits = down_splits(I, w->gate.format);
+  t.splits = splits;
   t.slots = M;
   t.h1 = h1_out;
   t.norm_w = norm_w;
@@ -616,6 +705,34 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
       return fail(MOEFFN_ERR_CUDA, "moe_plan_create: tensor map upload failed");
     }
   }
+  // Tensor maps of the grouped tensor-core GEMMs.
+  bool tc = true;
+  for (int e = 0; e < E && tc; ++e) tc = tc_ok(desc->experts[e]);
+  if (tc && p->has_shared) tc = tc_ok(*desc->shared);
+  if (tc) {
+    std::vector<TcMaps> tg(E), tu(E), td(E);
+    bool ok = true;
+    for (int e = 0; e < E && ok; ++e) {
+      ok = encode_tc_weight_maps(&tg[e], MOEFFN_Q_INT4_AFFINE_G32, g[e], Ie, H, 64) == cudaSuccess &&
+           encode_tc_weight_maps(&tu[e], MOEFFN_Q_INT4_AFFINE_G32, u[e], Ie, H, 64) == cudaSuccess &&
+           encode_tc_weight_maps(&td[e], MOEFFN_Q_INT4_AFFINE_G32, d[e], H, Ie, 128) == cudaSuccess;
+    }
+    if (ok && p->has_shared) {
+      ok = encode_tc_weight_maps(&p->tc_sg, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.gate), Is, H, 64) == cudaSuccess &&
+           encode_tc_weight_maps(&p->tc_su, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.up), Is, H, 64) == cudaSuccess &&
+           encode_tc_weight_maps(&p->tc_sd, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.down), H, Is, 128) == cudaSuccess;
+    }
+    const size_t bytes = sizeof(TcMaps) * E;
+    if (!ok || cudaMalloc(&p->d_tc_gate, bytes) != cudaSuccess || cudaMalloc(&p->d_tc_up, bytes) != cudaSuccess ||
+        cudaMalloc(&p->d_tc_down, bytes) != cudaSuccess ||
+        cudaMemcpy(p->d_tc_gate, tg.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(p->d_tc_up, tu.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(p->d_tc_down, td.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+      moe_plan_destroy(p);
+      return fail(MOEFFN_ERR_CUDA, "moe_plan_create: tensor-core GEMM maps failed");
+    }
+    p->tc = true;
+  }
   *plan = p;
   return MOEFFN_OK;
 }
@@ -627,6 +744,9 @@ int moe_plan_destroy(moeffn_moe_plan* plan) {
   cudaFree(plan->d_down);
   cudaFree(plan->d_maps);
   cudaFree(plan->d_maps_s);
+  cudaFree(plan->d_tc_gate);
+  cudaFree(plan->d_tc_up);
+  cudaFree(plan->d_tc_down);
   delete plan;
   return MOEFFN_OK;
 }
@@ -695,7 +815,85 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   const int splits = std::max(splits_r, splits_sh);
   const TmaGeom gu = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, H, max_tok);
   const TmaGeom dn = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 1, sp.ks_len, max_tok);
-  if (p->tma && gu.ok && dn.ok) {
+  int tc_splits_r = splits_r, tc_splits_s = splits_sh;
+  const bool use_tc = p->tc && M >= kTcMinMoeTokens && aligned16(x);
+  if (use_tc) {
+    // Token rows in pair-slot order feed phase 1's B operand.
+    GatherArgs ga{x, w.perm, k, H, P, w.xg};
+    {
+      ProfScope ps("gather_rows", s);
+      MOEFFN_CHECK_CUDA(launch_gather_rows(ga, s), "gather launch");
+    }
+    const int per_expert = std::max(1, P / std::min(E, P));
+    const int nt = tc_nt(std::min(per_expert, 128));
+    const int tt = (M + nt - 1) / nt;   // an expert has at most M token rows
+    TcGemmArgs g{};
+    g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
+    g.act = p->act;
+    g.mode = TC_GATEUP;
+    g.nt = nt;
+    g.N = Ie;
+    g.K = H;
+    g.Ns = Is;
+    g.Ks = H;
+    g.M = M;
+    g.offsets = w.offsets;
+    g.union_list = w.union_list;
+    g.n_union = w.n_union;
+    g.routed_jobs = routed_jobs;
+    g.slots = P;
+    g.tab0 = p->d_tc_gate;
+    g.tab1 = p->d_tc_up;
+    g.s0 = p->tc_sg;
+    g.s1 = p->tc_su;
+    g.out_act = w.acts;
+    g.out_act_s = w.acts_s;
+    g.ks_len = H;
+    g.token_tiles = tt;
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, w.xg, P, H, nt), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap_s, x, M, H, nt), "tensor map encode");
+    {
+      ProfScope ps("phase1_gateup_gemm_tc", s);
+      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (std::max(Ie, Is) + 63) / 64, 1, jobs, s), "phase-1 GEMM launch");
+    }
+    TcGemmArgs d{};
+    d.fmt = MOEFFN_Q_INT4_AFFINE_G32;
+    d.mode = TC_DOWN;
+    d.nt = nt;
+    d.N = H;
+    d.K = Ie;
+    d.Ns = H;
+    d.Ks = Is;
+    d.M = M;
+    d.offsets = w.offsets;
+    d.union_list = w.union_list;
+    d.n_union = w.n_union;
+    d.routed_jobs = routed_jobs;
+    d.slots = P;
+    d.tab0 = p->d_tc_down;
+    d.s0 = p->tc_sd;
+    d.out_d = w.d;
+    d.out_d_s = w.d_s;
+    d.token_tiles = tt;
+    const int row_tiles = (H + 127) / 128;
+    const int active = std::max(1, std::min(E, P)) * std::max(1, (per_expert + nt - 1) / nt);
+    const int want = (2 * kSMs + row_tiles * active - 1) / (row_tiles * active);
+    d.ks_len = tc_down_slice(Ie, MOEFFN_Q_INT4_AFFINE_G32, want, sp.routed);
+    tc_splits_r = (Ie + d.ks_len - 1) / d.ks_len;
+    tc_splits_s = Is > 0 ? (Is + d.ks_len - 1) / d.ks_len : 0;
+    if (tc_splits_s > sp.shared) {   // keep within the workspace's partial buffers
+      d.ks_len = sp.ks_len;
+      tc_splits_r = splits_r;
+      tc_splits_s = splits_sh;
+    }
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, P, Ie, nt), "tensor map encode");
+    if (Is > 0) MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap_s, w.acts_s, M, Is, nt), "tensor map encode");
+    {
+      ProfScope ps("phase2_down_gemm_tc", s);
+      MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, std::max(tc_splits_r, tc_splits_s), jobs, s),
+                        "phase-2 GEMM launch");
+    }
+  } else if (p->tma && gu.ok && dn.ok) {
     TmaGemvArgs g{};
     g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
     g.act = p->act;
@@ -829,10 +1027,10 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   t.M = M;
   t.N = H;
   t.d = w.d;
-  t.splits = splits_r;
+  t.splits = tc_splits_r;
   t.slots = P;
   t.d_s = p->has_shared ? w.d_s : nullptr;
-  t.splits_s = splits_sh;
+  t.splits_s = tc_splits_s;
   t.gate_logit = w.gate_logit;
   t.w = w.w;
   t.inv = w.inv;

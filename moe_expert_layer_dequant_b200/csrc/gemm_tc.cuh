@@ -1,0 +1,54 @@
+// Launch interface of the tcgen05 quantized GEMM (gemm_tc.cu).
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace moeffn {
+
+enum : int { TC_GATEUP = 2, TC_DOWN = 1 };
+
+// Tensor maps of one quantized matrix for the GEMM: codes (uint8, 128-byte
+// swizzled boxes of [rows][128 bytes]), INT4 scales and mins (u16 boxes of
+// [rows][8 groups]).
+struct TcMaps {
+  CUtensorMap codes, scale, mn;
+};
+
+struct TcGemmArgs {
+  CUtensorMap xmap;            // B operand rows (dense / routed jobs): bf16 [rows][K], boxes [NT][64]
+  CUtensorMap xmap_s;          // B operand rows of the shared job
+  TcMaps w0, w1;               // dense mode: gate, up (GATEUP) or down (w0)
+  const TcMaps* tab0;          // grouped mode: per expert [E]
+  const TcMaps* tab1;
+  TcMaps s0, s1;               // shared expert
+  const __half* rscale0;       // INT8 dense: per-row scales of w0 / w1
+  const __half* rscale1;
+  int fmt, act, mode, nt;
+  int N, K, Ns, Ks;            // dense / routed and shared shapes (rows, reduction)
+  int M;
+  const int* offsets;          // null: dense mode
+  const int* union_list;
+  const int* n_union;
+  int routed_jobs;
+  int slots;                   // slot count of the outputs (dense: M, grouped: M*topk)
+  uint16_t* out_act;           // GATEUP: [slots][N] bf16
+  uint16_t* out_act_s;         // [M][Ns]
+  float* out_d;                // DOWN: [splits][slots][N] fp32
+  float* out_d_s;              // [splits][M][N]
+  int ks_len;                  // K per split (multiple of the weight tile)
+  int token_tiles;             // grid.y = token_tiles * splits
+};
+
+// Rows of the weight tile per CTA: 64 features (gate and up stacked) or 128.
+inline int tc_rows_per_tile(int mode) { return mode == TC_GATEUP ? 64 : 128; }
+// K covered by one weight stage: 256 codes (INT4) or 128 (INT8).
+inline int tc_k_tile(int fmt) { return fmt == FMT_INT4_G32 ? 256 : 128; }
+
+size_t tc_gemm_smem(int fmt, int nt);
+cudaError_t encode_tc_weight_maps(TcMaps* m, int fmt, const QW& w, int N, int K, int box_rows);
+cudaError_t encode_tc_x_map(CUtensorMap* m, const uint16_t* x, int rows, int K, int nt);
+cudaError_t launch_tc_gemm(const TcGemmArgs& a, int row_tiles, int splits, int jobs, cudaStream_t s);
+unsigned int tc_gemm_fault_flags(bool clear);
+
+}  // namespace moeffn

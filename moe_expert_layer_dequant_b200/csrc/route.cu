@@ -166,7 +166,23 @@ __global__ void __launch_bounds__(1024) k_route(const RouteArgs a) {
   }
 }
 
+// Token rows in expert-grouped pair order: the B operand rows of the grouped
+// expert GEMMs. One CTA per slot, 16-byte copies.
+__global__ void __launch_bounds__(128) k_gather_rows(const GatherArgs a) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int s = blockIdx.x;
+  const int t = a.perm[s] / a.topk;
+  const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)t * a.H);
+  uint4* dst = reinterpret_cast<uint4*>(a.xg + (size_t)s * a.H);
+  for (int i = threadIdx.x; i < a.H / 8; i += blockDim.x) dst[i] = src[i];
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const GatherArgs& a, cudaStream_t s) {
+  return launch_pdl(k_gather_rows, dim3(a.P), dim3(128), 0, s, a);
+}
 
 cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t s) {
   const int rows = a.E + (a.w_sg != nullptr ? 1 : 0);

@@ -29,7 +29,16 @@ struct RouteArgs {
   int* n_union;                // [1] or null
 };
 
+// xg[s][:] = x[perm[s] / topk][:] for the P = M*topk pair slots (bf16 rows of H).
+struct GatherArgs {
+  const uint16_t* x;
+  const int* perm;
+  int topk, H, P;
+  uint16_t* xg;
+};
+
 cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t s);
+cudaError_t launch_gather_rows(const GatherArgs& a, cudaStream_t s);
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
 }  // namespace moeffn

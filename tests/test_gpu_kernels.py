@@ -122,6 +122,26 @@ def test_dense_small(cfg, shape, fmt, M):
     assert_bf16_close(dl.run(inp.x, zero), oracle.layer(inp), "h")
 
 
+# Token counts from 3 up run the tensor-core GEMM (tcgen05) where K allows:
+# token tiles of 16..256, several tiles and a ragged last tile.
+DENSE_TC = [
+    (2, dict(H=512, I=1280)),      # INT4-affine
+    (1, dict(H=256, I=640)),       # INT8-row
+    (2, dict(H=768, I=2304)),      # INT4, down split along K
+]
+
+
+@pytest.mark.parametrize("cfg,shape", DENSE_TC)
+@pytest.mark.parametrize("M", [3, 16, 40, 150, 300])
+def test_dense_tensor_core(cfg, shape, M):
+    c = synth.scaled_config(cfg, **shape)
+    inp = synth.make_inputs(c, M, 7)
+    dl = DeviceLayer(inp)
+    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "out")
+    inp.residual = np.zeros_like(inp.residual)
+    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "h")
+
+
 @pytest.mark.parametrize("shape", [dict(H=384, I=800), dict(H=256, I=2560)])   # the second splits K (INT8)
 @pytest.mark.parametrize("M", [1, 2, 3, 8])
 def test_shared_expert_small(M, shape):
@@ -142,7 +162,7 @@ MOE_SMALL = [
 
 
 @pytest.mark.parametrize("shape", MOE_SMALL)
-@pytest.mark.parametrize("M", [1, 2, 3, 7])
+@pytest.mark.parametrize("M", [1, 2, 3, 7, 9, 40])   # 9, 40: grouped tensor-core GEMMs where K allows
 def test_moe_small(shape, M):
     shape = dict(shape)
     c = synth.scaled_config(shape.pop("cfg"), **shape)
