@@ -7,15 +7,17 @@
 // the instruction. Per CTA: one tile of weight rows x one tile of tokens x the
 // job's K range (or one K split of it).
 //
-//  warp 0      producer: TMA loads of the quantized weight stages (codes in
-//              128-byte swizzled boxes, INT4 group scales and mins) and of the
-//              bf16 token tiles (128-byte swizzled, the MMA's B operand);
+//  warp 0      weight producer: TMA loads of the quantized weight stages
+//              (codes in 128-byte swizzled boxes, INT4 group scales and mins);
+//  warp 2      token producer: TMA loads of the bf16 token tiles (128-byte
+//              swizzled, the MMA's B operand);
 //  warp 1      allocates the TMEM accumulator and issues tcgen05.mma (one
 //              thread), releasing operand slots with tcgen05.commit;
-//  warps 4-7   dequantize: each thread owns one weight row and writes its 64
-//              bf16 weights of every K atom (w = RNE(q * scale + min), exact in
-//              fp32 before the rounding) into the swizzled canonical layout the
-//              MMA reads; then, as the epilogue, read TMEM (warp w%4 sees lanes
+//  warps 4-19  dequantize, in two groups of 8 warps taking alternate K atoms:
+//              two threads per weight row each write 32 bf16 weights of the
+//              atom (w = RNE(q * scale + min), exact in fp32 before the
+//              rounding) into the swizzled canonical layout the MMA reads;
+//  warps 4-7   then, as the epilogue, read TMEM (warp w%4 sees lanes
 //              32*(w%4)..+31) and write the outputs.
 //
 // Modes: GATEUP stacks 64 gate rows and the same 64 up rows in one 128-row A
@@ -33,9 +35,10 @@ namespace moeffn {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kSW = 2;                  // quantized weight stages
-constexpr int kSA = 4;                  // bf16 A atoms
+constexpr int kDqGroups = 2;            // dequant groups, taking alternate K atoms
+constexpr int kDqGroupWarps = 8;        // warps per group: two threads per weight row
+constexpr int kDqWarps = kDqGroups * kDqGroupWarps;   // warps 4..19
+constexpr int kThreads = 32 * (4 + kDqWarps);
 constexpr int kAtomBytes = 128 * 128;   // 128 rows x 64 bf16
 
 template <int FMT>
@@ -60,14 +63,16 @@ struct TcFmt<FMT_INT8_ROW> {
 template <int NT>
 struct TcTile {
   static constexpr int kSB = NT >= 256 ? 3 : 4;                 // B (token) atoms
+  static constexpr int kSW = NT <= 128 ? 4 : 2;                 // quantized weight stages
+  static constexpr int kSA = NT <= 32 ? 8 : (NT <= 64 ? 6 : 4); // bf16 A atoms
   static constexpr int kBBytes = NT * 128;
   static constexpr uint32_t kTmemCols = NT < 32 ? 32u : (uint32_t)NT;
 };
 
 template <int FMT, int NT>
 __host__ __device__ constexpr size_t tc_smem_bytes() {
-  return 1024 /*align slack*/ + 1024 /*barriers*/ + (size_t)kSW * TcFmt<FMT>::kStageBytes +
-         (size_t)kSA * kAtomBytes + (size_t)TcTile<NT>::kSB * TcTile<NT>::kBBytes;
+  return 1024 /*align slack*/ + 1024 /*barriers*/ + (size_t)TcTile<NT>::kSW * TcFmt<FMT>::kStageBytes +
+         (size_t)TcTile<NT>::kSA * kAtomBytes + (size_t)TcTile<NT>::kSB * TcTile<NT>::kBBytes;
 }
 
 struct Job {
@@ -105,56 +110,52 @@ __device__ __forceinline__ Job decode_job(const TcGemmArgs& a) {
 
 // ---- dequantization of one K atom (64 weights) of one row into the A tile ----
 
-// INT4: 64 codes = groups g0 = 2j, 2j+1 of the stage row (128-byte swizzled);
-// w = q * s + m in fp32 (exact), rounded to bf16.
-__device__ __forceinline__ void dequant_atom_int4(uint32_t wq, int r, int j, uint32_t a_atom) {
+// INT4: half hf of atom j is group g = 2j + hf of the stage row (one 16-byte
+// chunk of the 128-byte swizzled row, 32 codes); w = q * s + m in fp32
+// (exact), rounded to bf16, written as chunks 4hf..4hf+3 of the atom row.
+__device__ __forceinline__ void dequant_half_int4(uint32_t wq, int r, int j, int hf, uint32_t a_atom) {
   const uint32_t code_row = wq + r * 128;
-  const uint4 sc4 = lds_u128(wq + TcFmt<FMT_INT4_G32>::kCodeBytes + r * 16);
-  const uint4 mn4 = lds_u128(wq + TcFmt<FMT_INT4_G32>::kCodeBytes + TcFmt<FMT_INT4_G32>::kScaleBytes + r * 16);
-  const uint32_t scw[4] = {sc4.x, sc4.y, sc4.z, sc4.w}, mnw[4] = {mn4.x, mn4.y, mn4.z, mn4.w};
+  const int g = 2 * j + hf;
+  const uint32_t sw = lds_u32(wq + TcFmt<FMT_INT4_G32>::kCodeBytes + r * 16 + (g >> 1) * 4);
+  const uint32_t mw = lds_u32(wq + TcFmt<FMT_INT4_G32>::kCodeBytes + TcFmt<FMT_INT4_G32>::kScaleBytes + r * 16 + (g >> 1) * 4);
+  const float s = __half2float(__ushort_as_half((unsigned short)((sw >> ((g & 1) * 16)) & 0xFFFFu)));
+  const float m = __half2float(__ushort_as_half((unsigned short)((mw >> ((g & 1) * 16)) & 0xFFFFu)));
+  const uint4 cw = lds_u128(code_row + (((g ^ (r & 7)) & 7) << 4));
   const uint32_t arow = a_atom + r * 128;
   const uint32_t mg = kMagic, m0 = 0x000Fu, m1 = 0x00F0u, m2 = 0x0F00u, m3 = 0xF000u;
+  // The magic conversion leaves code i of a half-word scaled by 16^(i%4):
+  // undo it in the scale (exact powers of two).
+  const float2 s01 = make_float2(s, s * 0.0625f), s23 = make_float2(s * 0.00390625f, s * 0.000244140625f);
+  const float2 mm = make_float2(m, m), sub = make_float2(-kMagicF, -kMagicF);
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const int g = 2 * j + h;  // group within the stage row, also its 16-byte chunk
-    const uint4 cw = lds_u128(code_row + (((g ^ (r & 7)) & 7) << 4));
-    const uint32_t hs = (scw[g >> 1] >> ((g & 1) * 16)) & 0xFFFFu;
-    const uint32_t hm = (mnw[g >> 1] >> ((g & 1) * 16)) & 0xFFFFu;
-    const float s = __half2float(__ushort_as_half((unsigned short)hs));
-    const float m = __half2float(__ushort_as_half((unsigned short)hm));
-    // The magic conversion leaves code i of a half-word scaled by 16^(i%4):
-    // undo it in the scale (exact powers of two).
-    const float2 s01 = make_float2(s, s * 0.0625f), s23 = make_float2(s * 0.00390625f, s * 0.000244140625f);
-    const float2 mm = make_float2(m, m), sub = make_float2(-kMagicF, -kMagicF);
-    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t w = words[q], hi = w >> 16;
-      float2 c01 = make_float2(__uint_as_float(and_or(w, m0, mg)), __uint_as_float(and_or(w, m1, mg)));
-      float2 c23 = make_float2(__uint_as_float(and_or(w, m2, mg)), __uint_as_float(and_or(w, m3, mg)));
-      float2 c45 = make_float2(__uint_as_float(and_or(hi, m0, mg)), __uint_as_float(and_or(hi, m1, mg)));
-      float2 c67 = make_float2(__uint_as_float(and_or(hi, m2, mg)), __uint_as_float(and_or(hi, m3, mg)));
-      c01 = __ffma2_rn(__fadd2_rn(c01, sub), s01, mm);
-      c23 = __ffma2_rn(__fadd2_rn(c23, sub), s23, mm);
-      c45 = __ffma2_rn(__fadd2_rn(c45, sub), s01, mm);
-      c67 = __ffma2_rn(__fadd2_rn(c67, sub), s23, mm);
-      const uint4 out = make_uint4(pack_bf16x2(c01.x, c01.y), pack_bf16x2(c23.x, c23.y), pack_bf16x2(c45.x, c45.y),
-                                   pack_bf16x2(c67.x, c67.y));
-      const int chunk = 4 * h + q;  // 8 bf16 = 16 bytes of the 128-byte atom row
-      sts_u128(arow + ((chunk ^ (r & 7)) << 4), out);
-    }
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w = words[q], hi = w >> 16;
+    float2 c01 = make_float2(__uint_as_float(and_or(w, m0, mg)), __uint_as_float(and_or(w, m1, mg)));
+    float2 c23 = make_float2(__uint_as_float(and_or(w, m2, mg)), __uint_as_float(and_or(w, m3, mg)));
+    float2 c45 = make_float2(__uint_as_float(and_or(hi, m0, mg)), __uint_as_float(and_or(hi, m1, mg)));
+    float2 c67 = make_float2(__uint_as_float(and_or(hi, m2, mg)), __uint_as_float(and_or(hi, m3, mg)));
+    c01 = __ffma2_rn(__fadd2_rn(c01, sub), s01, mm);
+    c23 = __ffma2_rn(__fadd2_rn(c23, sub), s23, mm);
+    c45 = __ffma2_rn(__fadd2_rn(c45, sub), s01, mm);
+    c67 = __ffma2_rn(__fadd2_rn(c67, sub), s23, mm);
+    const uint4 out = make_uint4(pack_bf16x2(c01.x, c01.y), pack_bf16x2(c23.x, c23.y), pack_bf16x2(c45.x, c45.y),
+                                 pack_bf16x2(c67.x, c67.y));
+    const int chunk = 4 * hf + q;  // 8 bf16 = 16 bytes of the 128-byte atom row
+    sts_u128(arow + ((chunk ^ (r & 7)) << 4), out);
   }
 }
 
-// INT8: 64 signed codes (chunks 4j..4j+3 of the stage row) as exact bf16
-// integers; the row scale is applied in the epilogue.
-__device__ __forceinline__ void dequant_atom_int8(uint32_t wq, int r, int j, uint32_t a_atom) {
+// INT8: half hf of atom j is input chunks 4j+2hf, 4j+2hf+1 (32 signed codes)
+// as exact bf16 integers; the row scale is applied in the epilogue.
+__device__ __forceinline__ void dequant_half_int8(uint32_t wq, int r, int j, int hf, uint32_t a_atom) {
   const uint32_t code_row = wq + r * 128;
   const uint32_t arow = a_atom + r * 128;
   const uint32_t mg = kMagic;
   const float2 sub = make_float2(-(kMagicF + 128.0f), -(kMagicF + 128.0f));
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * hf + cc;                 // 16-code chunk within the atom
     const int chunk_in = 4 * j + c;
     const uint4 cw = lds_u128(code_row + (((chunk_in ^ (r & 7)) & 7) << 4));
     const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
@@ -204,21 +205,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   uint8_t* const gbase = smem_raw + (base - smem_addr(smem_raw));
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase);
   uint64_t* wq_full = bars;
-  uint64_t* wq_empty = wq_full + kSW;
-  uint64_t* a_full = wq_empty + kSW;
-  uint64_t* a_empty = a_full + kSA;
-  uint64_t* b_full = a_empty + kSA;
+  uint64_t* wq_empty = wq_full + T::kSW;
+  uint64_t* a_full = wq_empty + T::kSW;
+  uint64_t* a_empty = a_full + T::kSA;
+  uint64_t* b_full = a_empty + T::kSA;
   uint64_t* b_empty = b_full + T::kSB;
   uint64_t* acc_full = b_empty + T::kSB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + 512);
   const uint32_t wq_base = base + 1024;
-  const uint32_t a_base = wq_base + kSW * F::kStageBytes;
-  const uint32_t b_base = a_base + kSA * kAtomBytes;
+  const uint32_t a_base = wq_base + T::kSW * F::kStageBytes;
+  const uint32_t b_base = a_base + T::kSA * kAtomBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSW; ++i) { mbar_init(&wq_full[i], 1); mbar_init(&wq_empty[i], 4); }
-    for (int i = 0; i < kSA; ++i) { mbar_init(&a_full[i], 4); mbar_init(&a_empty[i], 1); }
+    for (int i = 0; i < T::kSW; ++i) { mbar_init(&wq_full[i], 1); mbar_init(&wq_empty[i], kDqWarps); }
+    for (int i = 0; i < T::kSA; ++i) { mbar_init(&a_full[i], kDqGroupWarps); mbar_init(&a_empty[i], 1); }
     for (int i = 0; i < T::kSB; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
     mbar_init(acc_full, 1);
     fence_mbar_init();
@@ -236,39 +237,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   const int row_tok = job.slot0 + t0;   // first B row (token or slot) of the tile
 
   if (warp == 0) {
-    // ---------------- producer ----------------
+    // ---------------- weight producer ----------------
+    // Runs up to kSW stages ahead of the dequantizers, independently of the
+    // token tiles, so the weight stream never waits on MMA progress.
     if (lane == 0) {
-      bool dead = false;
-      for (int k = 0; k < nk && !dead; ++k) {
-        if (k % F::kAtoms == 0) {
-          const int w = k / F::kAtoms, slot = w % kSW, use = w / kSW;
-          if (use > 0 && !mbar_wait(&wq_empty[slot], (use - 1) & 1)) { dead = true; break; }
-          const uint32_t st = wq_base + slot * F::kStageBytes;
-          uint8_t* gst = gbase + (st - base);
-          mbar_arrive_expect_tx(&wq_full[slot], F::kStageBytes);
-          const int kc = k0 + w * F::kKTile;                 // first K element of the stage
-          const int cx = (FMT == FMT_INT4_G32) ? kc / 2 : kc; // byte column of the codes
-          if (MODE == TC_GATEUP) {
-            tma_load_2d(gst, &job.m0->codes, cx, n0, &wq_full[slot]);
-            tma_load_2d(gst + 64 * 128, &job.m1->codes, cx, n0, &wq_full[slot]);
-            if (FMT == FMT_INT4_G32) {
-              uint8_t* gs = gst + F::kCodeBytes;
-              tma_load_2d(gs, &job.m0->scale, kc / 32, n0, &wq_full[slot]);
-              tma_load_2d(gs + 64 * 16, &job.m1->scale, kc / 32, n0, &wq_full[slot]);
-              tma_load_2d(gs + F::kScaleBytes, &job.m0->mn, kc / 32, n0, &wq_full[slot]);
-              tma_load_2d(gs + F::kScaleBytes + 64 * 16, &job.m1->mn, kc / 32, n0, &wq_full[slot]);
-            }
-          } else {
-            tma_load_2d(gst, &job.m0->codes, cx, n0, &wq_full[slot]);
-            if (FMT == FMT_INT4_G32) {
-              uint8_t* gs = gst + F::kCodeBytes;
-              tma_load_2d(gs, &job.m0->scale, kc / 32, n0, &wq_full[slot]);
-              tma_load_2d(gs + F::kScaleBytes, &job.m0->mn, kc / 32, n0, &wq_full[slot]);
-            }
+      const int nw = nk / F::kAtoms;
+      for (int w = 0; w < nw; ++w) {
+        const int slot = w % T::kSW, use = w / T::kSW;
+        if (use > 0 && !mbar_wait_spin(&wq_empty[slot], (use - 1) & 1)) break;
+        const uint32_t st = wq_base + slot * F::kStageBytes;
+        uint8_t* gst = gbase + (st - base);
+        mbar_arrive_expect_tx(&wq_full[slot], F::kStageBytes);
+        const int kc = k0 + w * F::kKTile;                 // first K element of the stage
+        const int cx = (FMT == FMT_INT4_G32) ? kc / 2 : kc; // byte column of the codes
+        if (MODE == TC_GATEUP) {
+          tma_load_2d(gst, &job.m0->codes, cx, n0, &wq_full[slot]);
+          tma_load_2d(gst + 64 * 128, &job.m1->codes, cx, n0, &wq_full[slot]);
+          if (FMT == FMT_INT4_G32) {
+            uint8_t* gs = gst + F::kCodeBytes;
+            tma_load_2d(gs, &job.m0->scale, kc / 32, n0, &wq_full[slot]);
+            tma_load_2d(gs + 64 * 16, &job.m1->scale, kc / 32, n0, &wq_full[slot]);
+            tma_load_2d(gs + F::kScaleBytes, &job.m0->mn, kc / 32, n0, &wq_full[slot]);
+            tma_load_2d(gs + F::kScaleBytes + 64 * 16, &job.m1->mn, kc / 32, n0, &wq_full[slot]);
+          }
+        } else {
+          tma_load_2d(gst, &job.m0->codes, cx, n0, &wq_full[slot]);
+          if (FMT == FMT_INT4_G32) {
+            uint8_t* gs = gst + F::kCodeBytes;
+            tma_load_2d(gs, &job.m0->scale, kc / 32, n0, &wq_full[slot]);
+            tma_load_2d(gs + F::kScaleBytes, &job.m0->mn, kc / 32, n0, &wq_full[slot]);
           }
         }
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------- token-tile producer ----------------
+    if (lane == 0) {
+      for (int k = 0; k < nk; ++k) {
         const int slot = k % T::kSB, use = k / T::kSB;
-        if (use > 0 && !mbar_wait(&b_empty[slot], (use - 1) & 1)) { dead = true; break; }
+        if (use > 0 && !mbar_wait_spin(&b_empty[slot], (use - 1) & 1)) break;
         mbar_arrive_expect_tx(&b_full[slot], T::kBBytes);
         tma_load_2d(gbase + (b_base - base) + slot * T::kBBytes, job.xmap, k0 + k * 64, row_tok, &b_full[slot]);
       }
@@ -279,8 +286,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
       constexpr uint32_t idesc = idesc_bf16_f32(128, NT);
       bool dead = false;
       for (int k = 0; k < nk; ++k) {
-        const int as = k % kSA, bs = k % T::kSB;
-        if (!mbar_wait(&a_full[as], (k / kSA) & 1) || !mbar_wait(&b_full[bs], (k / T::kSB) & 1)) {
+        const int as = k % T::kSA, bs = k % T::kSB;
+        if (!mbar_wait_spin(&a_full[as], (k / T::kSA) & 1) || !mbar_wait_spin(&b_full[bs], (k / T::kSB) & 1)) {
           dead = true;
           break;
         }
@@ -296,26 +303,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
       if (!dead) umma_commit(acc_full);
     }
   } else if (warp >= 4) {
-    // ---------------- dequantize, then epilogue ----------------
-    const int r = threadIdx.x - 128;    // weight row of the A tile = TMEM lane
+    // ---------------- dequantize (warps 4-19), then epilogue (warps 4-7) ----------------
+    // Two groups of 8 warps take alternate K atoms, so that one group's store
+    // drain and barrier release overlap the other's conversion. Every A slot
+    // belongs to one group (the ring depth is even).
+    const int grp = (warp - 4) / kDqGroupWarps;
+    const int tg = (warp - 4 - grp * kDqGroupWarps) * 32 + lane;
+    const int r = tg & 127, hf = tg >> 7;   // weight row of the A tile, half of the atom row
     bool dead = false;
-    for (int k = 0; k < nk; ++k) {
-      const int w = k / F::kAtoms, j = k % F::kAtoms, ws = w % kSW;
-      const int as = k % kSA, ause = k / kSA;
-      if (!dead && j == 0 && !mbar_wait(&wq_full[ws], (w / kSW) & 1)) dead = true;
-      if (!dead && ause > 0 && !mbar_wait(&a_empty[as], (ause - 1) & 1)) dead = true;
+    for (int k = grp; k < nk; k += kDqGroups) {
+      const int w = k / F::kAtoms, j = k % F::kAtoms, ws = w % T::kSW;
+      const int as = k % T::kSA, ause = k / T::kSA;
+      if (!dead && j < kDqGroups && !mbar_wait_spin(&wq_full[ws], (w / T::kSW) & 1)) dead = true;
+      if (!dead && ause > 0 && !mbar_wait_spin(&a_empty[as], (ause - 1) & 1)) dead = true;
       if (!dead) {
         const uint32_t wq = wq_base + ws * F::kStageBytes;
-        if (FMT == FMT_INT4_G32) dequant_atom_int4(wq, r, j, a_base + as * kAtomBytes);
-        else dequant_atom_int8(wq, r, j, a_base + as * kAtomBytes);
+        if (FMT == FMT_INT4_G32) dequant_half_int4(wq, r, j, hf, a_base + as * kAtomBytes);
+        else dequant_half_int8(wq, r, j, hf, a_base + as * kAtomBytes);
       }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&a_full[as]);
-        if (j == F::kAtoms - 1) mbar_arrive(&wq_empty[ws]);
+        if (j >= F::kAtoms - kDqGroups) mbar_arrive(&wq_empty[ws]);   // the group's last atom of the stage
       }
     }
+    if (warp >= 8) goto done;   // the epilogue is one warpgroup (TMEM lane quarters 0-3)
     // Epilogue: TMEM lanes = tile rows, columns = tokens.
     if (!dead && !mbar_wait(acc_full, 0)) dead = true;
     dead = __any_sync(0xffffffffu, dead);   // TMEM loads are warp-collective
@@ -382,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
     }
     tc_fence_before();
   }
+done:
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -419,7 +433,9 @@ cudaError_t launch_nt(const TcGemmArgs& a, dim3 grid, cudaStream_t s) {
 size_t tc_gemm_smem(int fmt, int nt) {
   const size_t stage = fmt == FMT_INT4_G32 ? TcFmt<FMT_INT4_G32>::kStageBytes : TcFmt<FMT_INT8_ROW>::kStageBytes;
   const int sb = nt >= 256 ? 3 : 4;
-  return 2048 + kSW * stage + (size_t)kSA * kAtomBytes + (size_t)sb * nt * 128;
+  const int sw = nt <= 128 ? 4 : 2;
+  const int sa = nt <= 32 ? 8 : (nt <= 64 ? 6 : 4);
+  return 2048 + sw * stage + (size_t)sa * kAtomBytes + (size_t)sb * nt * 128;
 }
 
 cudaError_t encode_tc_weight_maps(TcMaps* m, int fmt, const QW& w, int N, int K, int box_rows) {

@@ -69,11 +69,57 @@ __device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
-// One CTA. Each warp selects the top-k of its tokens: every lane holds E/32
-// logits; k rounds of a warp-wide arg-max, the winner's lane retires it.
-// Weights: softmax over the k selected logits times the per-expert scale
-// (ones), rounded to fp16. Then the stable expert-grouped order of the pairs
-// p = t*k + r (counts, offsets, union, placement by warp 0).
+// Top-k of one token by one warp: every lane holds up to PL logits (experts
+// lane, lane+32, ...); k rounds of a warp-wide arg-max, the winner's lane
+// retires it. Weights: softmax over the k selected logits times the
+// per-expert scale (ones), rounded to fp16.
+template <int PL>
+__device__ __forceinline__ void topk_token(const RouteArgs& a, int t, int lane) {
+  const float* l = a.logits + (size_t)t * a.E;
+  float lv[PL];
+  unsigned taken = 0;
+#pragma unroll
+  for (int j = 0; j < PL; ++j) {
+    const int e = lane + 32 * j;
+    lv[j] = e < a.E ? l[e] : 0.f;
+  }
+  float top0 = 0.f, zsum = 0.f;
+  float zr[kMaxTopK];
+  int ir[kMaxTopK];
+  for (int r = 0; r < a.k; ++r) {
+    float bv = -INFINITY;   // lanes without a candidate never win
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < PL; ++j) {
+      const int e = lane + 32 * j;
+      if (e < a.E && !((taken >> j) & 1u) && beats(lv[j], e, bv, bi)) {
+        bv = lv[j];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (beats(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (r == 0) top0 = bv;
+    zr[r] = expf(bv - top0);
+    ir[r] = bi;
+    zsum += zr[r];
+  }
+  if (lane == 0) {
+    for (int r = 0; r < a.k; ++r) {
+      a.idx[t * a.k + r] = ir[r];
+      a.w[t * a.k + r] = __half2float(__float2half_rn(zr[r] / zsum));
+    }
+  }
+}
+
+// One CTA: a warp per token for the top-k, then the stable expert-grouped
+// order of the pairs p = t*k + r (counts, offsets, union, placement by warp 0).
+template <int PL>
 __global__ void __launch_bounds__(1024) k_route(const RouteArgs a) {
   extern __shared__ int sm[];
   pdl_launch_dependents();
@@ -83,50 +129,8 @@ __global__ void __launch_bounds__(1024) k_route(const RouteArgs a) {
   int* offs = sm + 2 * a.E;         // [E+1]
   const int P = a.M * a.k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-  const int per_lane = (a.E + 31) / 32;
 
-  for (int t = warp; t < a.M; t += nwarps) {
-    const float* l = a.logits + (size_t)t * a.E;
-    float lv[kMaxExperts / 32];
-    unsigned taken = 0;
-#pragma unroll
-    for (int j = 0; j < kMaxExperts / 32; ++j) {
-      const int e = lane + 32 * j;
-      lv[j] = (j < per_lane && e < a.E) ? l[e] : 0.f;
-    }
-    float top0 = 0.f, zsum = 0.f;
-    float zr[kMaxTopK];
-    int ir[kMaxTopK];
-    for (int r = 0; r < a.k; ++r) {
-      float bv = -INFINITY;   // lanes without a candidate never win
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int j = 0; j < kMaxExperts / 32; ++j) {
-        const int e = lane + 32 * j;
-        if (j < per_lane && e < a.E && !((taken >> j) & 1u) && beats(lv[j], e, bv, bi)) {
-          bv = lv[j];
-          bi = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (beats(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (r == 0) top0 = bv;
-      zr[r] = expf(bv - top0);
-      ir[r] = bi;
-      zsum += zr[r];
-    }
-    if (lane == 0) {
-      for (int r = 0; r < a.k; ++r) {
-        a.idx[t * a.k + r] = ir[r];
-        a.w[t * a.k + r] = __half2float(__float2half_rn(zr[r] / zsum));
-      }
-    }
-  }
+  for (int t = warp; t < a.M; t += nwarps) topk_token<PL>(a, t, lane);
   for (int e = threadIdx.x; e < a.E; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
   __syncthreads();
   if (a.perm == nullptr) return;
@@ -192,7 +196,12 @@ cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t s) {
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)(3 * a.E + 1) * sizeof(int);
   const int threads = std::min(1024, std::max(128, a.M * 32));   // a warp per token
-  return launch_pdl(k_route, dim3(1), dim3(threads), smem, s, a);
+  const int pl = (a.E + 31) / 32;
+  if (pl <= 1) return launch_pdl(k_route<1>, dim3(1), dim3(threads), smem, s, a);
+  if (pl <= 2) return launch_pdl(k_route<2>, dim3(1), dim3(threads), smem, s, a);
+  if (pl <= 4) return launch_pdl(k_route<4>, dim3(1), dim3(threads), smem, s, a);
+  if (pl <= 8) return launch_pdl(k_route<8>, dim3(1), dim3(threads), smem, s, a);
+  return launch_pdl(k_route<32>, dim3(1), dim3(threads), smem, s, a);
 }
 
 }  // namespace moeffn
