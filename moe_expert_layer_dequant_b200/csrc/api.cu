@@ -155,22 +155,17 @@ int mt_for(int tokens) { return tokens <= 1 ? 1 : 2; }
 
 // ---- tensor-core GEMM eligibility and geometry ------------------------------
 
-constexpr int kTcMinTokens = 3;      // dense: token rows from which the GEMM replaces the GEMV
+constexpr int kTcMinTokens = 6;      // dense: token rows from which the GEMM replaces the GEMV
 constexpr int kTcMinMoeTokens = 8;   // MoE layer: token rows from which the grouped GEMMs are used
 
+// Rows a multiple of 16 keep every 8-column output chunk of the epilogue
+// inside the matrix and 16-byte aligned.
 bool tc_ok(const moeffn_qweight& w) {
-  if (!aligned16(w.q)) return false;
+  if (!aligned16(w.q) || w.rows % 16 != 0) return false;
   if (w.format == MOEFFN_Q_INT4_AFFINE_G32) return w.cols % 256 == 0 && aligned16(w.scale) && aligned16(w.min);
-  return w.format == MOEFFN_Q_INT8_ROW && w.cols % 128 == 0;
+  return w.format == MOEFFN_Q_INT8_ROW && w.cols % 128 == 0 && aligned16(w.scale);
 }
 bool tc_ok(const moeffn_ffn& f) { return tc_ok(f.gate) && tc_ok(f.up) && tc_ok(f.down); }
-
-// Token tile (MMA N) for an expected number of token rows per weight matrix.
-int tc_nt(int tokens) {
-  int nt = 16;
-  while (nt < tokens && nt < 256) nt *= 2;
-  return nt;
-}
 
 // K split of a down-projection GEMM: about `want` splits, at most `max_splits`,
 // slices a multiple of the weight stage K.
@@ -288,12 +283,14 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
                   cudaStream_t s, int* splits_out) {
   const int fmt = f.gate.format;
   if (M >= kTcMinTokens && tc_ok(f) && aligned16(x)) {
-    const int nt = tc_nt(M), tt = (M + nt - 1) / nt;
+    const int mt = tc_mt_for(M), tpc = tc_tokens_per_cta(mt), tt = (M + tpc - 1) / tpc;
+    const int fg = tc_gateup_feat(I), rd = tc_down_rows(H);
     TcGemmArgs g{};
     g.fmt = fmt;
     g.act = act;
     g.mode = TC_GATEUP;
-    g.nt = nt;
+    g.mt = mt;
+    g.tile = fg;
     g.N = I;
     g.K = H;
     g.M = M;
@@ -303,17 +300,18 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     g.token_tiles = tt;
     g.rscale0 = static_cast<const __half*>(f.gate.scale);
     g.rscale1 = static_cast<const __half*>(f.up.scale);
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, x, M, H, nt), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w0, fmt, to_qw(f.gate), I, H, 64), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w1, fmt, to_qw(f.up), I, H, 64), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, x, M, H), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w0, fmt, to_qw(f.gate), I, H, fg), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w1, fmt, to_qw(f.up), I, H, fg), "tensor map encode");
     {
       ProfScope ps("gateup_gemm_tc", s);
-      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (I + 63) / 64, 1, 1, s), "gate/up GEMM launch");
+      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (I + fg - 1) / fg, 1, 1, s), "gate/up GEMM launch");
     }
     TcGemmArgs d{};
     d.fmt = fmt;
     d.mode = TC_DOWN;
-    d.nt = nt;
+    d.mt = mt;
+    d.tile = rd;
     d.N = H;
     d.K = I;
     d.M = M;
@@ -321,12 +319,12 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.out_d = w.d;
     d.token_tiles = tt;
     d.rscale0 = static_cast<const __half*>(f.down.scale);
-    const int row_tiles = (H + 127) / 128;
+    const int row_tiles = (H + rd - 1) / rd;
     const int want = (kSMs + row_tiles * tt - 1) / (row_tiles * tt);
     d.ks_len = tc_down_slice(I, fmt, want, down_splits_any(I));
     const int splits = (I + d.ks_len - 1) / d.ks_len;
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, M, I, nt), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&d.w0, fmt, to_qw(f.down), H, I, 128), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, M, I), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&d.w0, fmt, to_qw(f.down), H, I, rd), "tensor map encode");
     {
       ProfScope ps("down_gemm_tc", s);
       MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, splits, 1, s), "down GEMM launch");
@@ -444,10 +442,11 @@ struct moeffn_moe_plan {
   QWMaps* d_maps = nullptr;    // [E] tensor maps of the expert down matrices (K split)
   QWMaps* d_maps_s = nullptr;  // [1] shared expert down (K split)
   bool tc = false;             // tensor-core GEMM maps built
-  TcMaps* d_tc_gate = nullptr; // [E] (64-row boxes)
-  TcMaps* d_tc_up = nullptr;   // [E] (64-row boxes)
-  TcMaps* d_tc_down = nullptr; // [E] (128-row boxes)
-  TcMaps tc_sg{}, tc_su{}, tc_sd{};
+  TcMaps* d_tc_gate = nullptr; // [E] (boxes of tc_fe rows)
+  TcMaps* d_tc_up = nullptr;   // [E] (boxes of tc_fe rows)
+  TcMaps* d_tc_down = nullptr; // [E] (boxes of tc_rd rows)
+  TcMaps tc_sg{}, tc_su{}, tc_sd{};   // shared expert (tc_fs, tc_fs, tc_rd rows)
+  int tc_fe = 0, tc_fs = 0, tc_rd = 0; // GATEUP features per tile (routed, shared), DOWN rows per tile
 };
 
 extern "C" {
@@ -711,16 +710,20 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   if (tc && p->has_shared) tc = tc_ok(*desc->shared);
   if (tc) {
     std::vector<TcMaps> tg(E), tu(E), td(E);
+    p->tc_fe = tc_gateup_feat(Ie);
+    p->tc_fs = p->has_shared ? tc_gateup_feat(Is) : 8;
+    p->tc_rd = tc_down_rows(H);
+    const int fe = p->tc_fe, fs = p->tc_fs, rd = p->tc_rd;
     bool ok = true;
     for (int e = 0; e < E && ok; ++e) {
-      ok = encode_tc_weight_maps(&tg[e], MOEFFN_Q_INT4_AFFINE_G32, g[e], Ie, H, 64) == cudaSuccess &&
-           encode_tc_weight_maps(&tu[e], MOEFFN_Q_INT4_AFFINE_G32, u[e], Ie, H, 64) == cudaSuccess &&
-           encode_tc_weight_maps(&td[e], MOEFFN_Q_INT4_AFFINE_G32, d[e], H, Ie, 128) == cudaSuccess;
+      ok = encode_tc_weight_maps(&tg[e], MOEFFN_Q_INT4_AFFINE_G32, g[e], Ie, H, fe) == cudaSuccess &&
+           encode_tc_weight_maps(&tu[e], MOEFFN_Q_INT4_AFFINE_G32, u[e], Ie, H, fe) == cudaSuccess &&
+           encode_tc_weight_maps(&td[e], MOEFFN_Q_INT4_AFFINE_G32, d[e], H, Ie, rd) == cudaSuccess;
     }
     if (ok && p->has_shared) {
-      ok = encode_tc_weight_maps(&p->tc_sg, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.gate), Is, H, 64) == cudaSuccess &&
-           encode_tc_weight_maps(&p->tc_su, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.up), Is, H, 64) == cudaSuccess &&
-           encode_tc_weight_maps(&p->tc_sd, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.down), H, Is, 128) == cudaSuccess;
+      ok = encode_tc_weight_maps(&p->tc_sg, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.gate), Is, H, fs) == cudaSuccess &&
+           encode_tc_weight_maps(&p->tc_su, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.up), Is, H, fs) == cudaSuccess &&
+           encode_tc_weight_maps(&p->tc_sd, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.down), H, Is, rd) == cudaSuccess;
     }
     const size_t bytes = sizeof(TcMaps) * E;
     if (!ok || cudaMalloc(&p->d_tc_gate, bytes) != cudaSuccess || cudaMalloc(&p->d_tc_up, bytes) != cudaSuccess ||
@@ -824,14 +827,20 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
       ProfScope ps("gather_rows", s);
       MOEFFN_CHECK_CUDA(launch_gather_rows(ga, s), "gather launch");
     }
+    // One CTA should cover a whole expert's token rows, since a second CTA
+    // would dequantize every weight of the expert again: two 128-row token
+    // tiles per CTA once the expected load, plus half again for the routing
+    // spread, passes 128.
     const int per_expert = std::max(1, P / std::min(E, P));
-    const int nt = tc_nt(std::min(per_expert, 128));
-    const int tt = (M + nt - 1) / nt;   // an expert has at most M token rows
+    const int mt = tc_mt_for(per_expert + per_expert / 2), tpc = tc_tokens_per_cta(mt);
+    const int tt = (M + tpc - 1) / tpc;   // an expert has at most M token rows
     TcGemmArgs g{};
     g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
     g.act = p->act;
     g.mode = TC_GATEUP;
-    g.nt = nt;
+    g.mt = mt;
+    g.tile = p->tc_fe;
+    g.tile_s = p->tc_fs;
     g.N = Ie;
     g.K = H;
     g.Ns = Is;
@@ -850,16 +859,19 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     g.out_act_s = w.acts_s;
     g.ks_len = H;
     g.token_tiles = tt;
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, w.xg, P, H, nt), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap_s, x, M, H, nt), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, w.xg, P, H), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap_s, x, M, H), "tensor map encode");
+    const int rt1 = std::max((Ie + p->tc_fe - 1) / p->tc_fe, Is > 0 ? (Is + p->tc_fs - 1) / p->tc_fs : 0);
     {
       ProfScope ps("phase1_gateup_gemm_tc", s);
-      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (std::max(Ie, Is) + 63) / 64, 1, jobs, s), "phase-1 GEMM launch");
+      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, rt1, 1, jobs, s), "phase-1 GEMM launch");
     }
     TcGemmArgs d{};
     d.fmt = MOEFFN_Q_INT4_AFFINE_G32;
     d.mode = TC_DOWN;
-    d.nt = nt;
+    d.mt = mt;
+    d.tile = p->tc_rd;
+    d.tile_s = p->tc_rd;
     d.N = H;
     d.K = Ie;
     d.Ns = H;
@@ -875,8 +887,8 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     d.out_d = w.d;
     d.out_d_s = w.d_s;
     d.token_tiles = tt;
-    const int row_tiles = (H + 127) / 128;
-    const int active = std::max(1, std::min(E, P)) * std::max(1, (per_expert + nt - 1) / nt);
+    const int row_tiles = (H + p->tc_rd - 1) / p->tc_rd;
+    const int active = std::max(1, std::min(E, P)) * std::max(1, (per_expert + tpc - 1) / tpc);
     const int want = (2 * kSMs + row_tiles * active - 1) / (row_tiles * active);
     d.ks_len = tc_down_slice(Ie, MOEFFN_Q_INT4_AFFINE_G32, want, sp.routed);
     tc_splits_r = (Ie + d.ks_len - 1) / d.ks_len;
@@ -886,8 +898,8 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
       tc_splits_r = splits_r;
       tc_splits_s = splits_sh;
     }
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, P, Ie, nt), "tensor map encode");
-    if (Is > 0) MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap_s, w.acts_s, M, Is, nt), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, P, Ie), "tensor map encode");
+    if (Is > 0) MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap_s, w.acts_s, M, Is), "tensor map encode");
     {
       ProfScope ps("phase2_down_gemm_tc", s);
       MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, std::max(tc_splits_r, tc_splits_s), jobs, s),
