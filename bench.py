@@ -307,10 +307,14 @@ def run_ours(args, rank, world, local_rank):
         weight_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
         # dominant kernel: largest share of device time in the profiled pass
         dom_name, (dom_n, dom_ms) = max(prof.items(), key=lambda kv: kv[1][1])
-        role = "gateup" if "gateup" in dom_name else ("down" if "down" in dom_name else None)
+        fl = algorithmic_flops(c, M)
+        fl["total"] = fl["gateup"] + fl["down"]
+        # the single-stream FFN kernel reads every weight of the layer
+        role = ("total" if "ffn_stream" in dom_name else
+                "gateup" if "gateup" in dom_name else ("down" if "down" in dom_name else None))
         dom_bytes = ab[role] if role else None
         dom_avg_s = dom_ms / dom_n * 1e-3
-        dom_flops = algorithmic_flops(c, M)[role] if role else None
+        dom_flops = fl[role] if role else None
         # bound: the larger of the weight-stream time and the tensor-core time
         tensor_bound = bool(dom_flops and "gemm_tc" in dom_name and bf16_tf > 0 and
                             dom_flops / (bf16_tf * 1e12) > dom_bytes / (hbm * 1e9))

@@ -19,6 +19,7 @@
 //  shared job  : the MoE layer's shared expert over all M tokens.
 // A CTA takes a contiguous range of the job's rows (a multiple of R rows).
 #include "gemv_tma.cuh"
+#include "gemv_math.cuh"
 #include "sync.cuh"
 #include "tmap.cuh"
 #include "launch.cuh"
@@ -26,71 +27,6 @@
 namespace moeffn {
 
 namespace {
-
-// Activations are staged per 16-byte weight chunk as int16 fixed point with one
-// power-of-two factor per chunk: x = xi * 2^(e-14), e = floor(log2(max|x|)).
-// A bf16 value has 8 significant bits, so every value within 2^7 of the
-// chunk's largest is exact and the rest lose only bits below 2^(e-15).
-// Codes times xi are then summed exactly in int32 with DP2A (two 16x8-bit
-// products per instruction) and scaled once per chunk.
-__device__ __forceinline__ int dp2a_lo_u(int a, uint32_t b, int c) {
-  int d;
-  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ int dp2a_hi_u(int a, uint32_t b, int c) {
-  int d;
-  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ int dp2a_lo_s(int a, uint32_t b, int c) {
-  int d;
-  asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ int dp2a_hi_s(int a, uint32_t b, int c) {
-  int d;
-  asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-template <int FMT>
-struct Codes;
-
-// INT4: a chunk is one group of 32 codes (4 words). Word codes q0..q7: the
-// low nibbles of its bytes are q0,q2,q4,q6 and the high nibbles q1,q3,q5,q7,
-// so the staged int16 of a word are ordered x0,x2,x4,x6,x1,x3,x5,x7.
-template <>
-struct Codes<FMT_INT4_G32> {
-  static constexpr int kChunk = 32;
-  static constexpr int kStageBytes = 80;  // 64 bytes of int16 + 16 bytes pad (bank spread)
-  static __device__ __forceinline__ int slot_of(int j) {  // position of element j of a word
-    return (j & 1) * 4 + (j >> 1);
-  }
-  // Adds the 8 products of word w with its staged activations (16 bytes).
-  static __device__ __forceinline__ void dot_word(uint32_t w, uint4 x, int& p0, int& p1) {
-    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-    p0 = dp2a_lo_u((int)x.x, lo, p0);
-    p1 = dp2a_hi_u((int)x.y, lo, p1);
-    p0 = dp2a_lo_u((int)x.z, hi, p0);
-    p1 = dp2a_hi_u((int)x.w, hi, p1);
-  }
-};
-
-// INT8: a chunk is 16 signed codes (4 words); staged in natural order.
-template <>
-struct Codes<FMT_INT8_ROW> {
-  static constexpr int kChunk = 16;
-  static constexpr int kStageBytes = 48;  // 32 bytes of int16 + 16 bytes pad
-  static __device__ __forceinline__ int slot_of(int j) { return j; }
-  // Two words (8 codes) with their staged activations (16 bytes).
-  static __device__ __forceinline__ void dot_word(uint32_t w0, uint32_t w1, uint4 x, int& p0, int& p1) {
-    p0 = dp2a_lo_s((int)x.x, w0, p0);
-    p1 = dp2a_hi_s((int)x.y, w0, p1);
-    p0 = dp2a_lo_s((int)x.z, w1, p0);
-    p1 = dp2a_hi_s((int)x.w, w1, p1);
-  }
-};
 
 struct Job {
   QW m[2];
@@ -252,45 +188,12 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
     // the chunk's power-of-two factor and (INT4) its plain sum; zero pad rows.
     for (int i = threadIdx.x; i < tok_rows * nch; i += nthreads) {
       const int r = i / nch, c = i - r * nch;
-      uint16_t v[C::kChunk];
+      const uint16_t* p = nullptr;
       if (r < tn) {
         const int row = job.gather ? a.perm[job.slot0 + tb + r] / a.topk : job.slot0 + tb + r;
-        const uint4* p = reinterpret_cast<const uint4*>(src + (size_t)row * ld + k0 + c * C::kChunk);
-#pragma unroll
-        for (int q = 0; q < C::kChunk / 8; ++q) {
-          const uint4 u = p[q];
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            v[8 * q + 2 * j] = (uint16_t)(w[j] & 0xFFFFu);
-            v[8 * q + 2 * j + 1] = (uint16_t)(w[j] >> 16);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < C::kChunk; ++j) v[j] = 0;
+        p = src + (size_t)row * ld + k0 + c * C::kChunk;
       }
-      float amax = 0.f, sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < C::kChunk; ++j) {
-        const float f = bf16_bits_to_float(v[j]);
-        amax = fmaxf(amax, fabsf(f));
-        sum += f;
-      }
-      int e = 0;
-      if (amax > 0.f) {
-        frexpf(amax, &e);
-        e -= 1;                                   // amax in [2^e, 2^(e+1))
-      }
-      int16_t* dst = reinterpret_cast<int16_t*>(xi + r * tok_stride + c * C::kStageBytes);
-      constexpr int kW = (C::kChunk == 32 ? 8 : 4);   // codes per 32-bit word
-#pragma unroll
-      for (int j = 0; j < C::kChunk; ++j) {
-        const float f = bf16_bits_to_float(v[j]);
-        dst[(j / kW) * kW + C::slot_of(j % kW)] = (int16_t)(amax > 0.f ? __float2int_rn(ldexpf(f, 14 - e)) : 0);
-      }
-      xf[r * nch + c] = amax > 0.f ? ldexpf(1.0f, e - 14) : 0.f;
-      if (kInt4) xsum[r * nch + c] = sum;
+      stage_chunk<FMT>(p, xi + r * tok_stride + c * C::kStageBytes, &xf[r * nch + c], &xsum[r * nch + c]);
     }
     consumer_sync(nthreads);
 
