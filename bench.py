@@ -309,9 +309,7 @@ def run_ours(args, rank, world, local_rank):
         dom_name, (dom_n, dom_ms) = max(prof.items(), key=lambda kv: kv[1][1])
         fl = algorithmic_flops(c, M)
         fl["total"] = fl["gateup"] + fl["down"]
-        # the single-stream FFN kernel reads every weight of the layer
-        role = ("total" if "ffn_stream" in dom_name else
-                "gateup" if "gateup" in dom_name else ("down" if "down" in dom_name else None))
+        role = "gateup" if "gateup" in dom_name else ("down" if "down" in dom_name else None)
         dom_bytes = ab[role] if role else None
         dom_avg_s = dom_ms / dom_n * 1e-3
         dom_flops = fl[role] if role else None

@@ -9,7 +9,6 @@
 #include "../../include/moeffn.h"
 #include "common.cuh"
 #include "gemv.cuh"
-#include "ffn_stream.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_tma.cuh"
 #include "tmap.cuh"
@@ -456,7 +455,7 @@ const char* moeffn_last_error(void) { return g_last_error.c_str(); }
 
 unsigned int moeffn_device_faults(int clear) {
   // Blocking read of the kernels' fault words (bounded waits that ran out).
-  return tma_gemv_fault_flags(clear != 0) | tc_gemm_fault_flags(clear != 0) | ffn_stream_fault_flags(clear != 0);
+  return tma_gemv_fault_flags(clear != 0) | tc_gemm_fault_flags(clear != 0);
 }
 
 size_t moeffn_workspace_bytes(int kind, int M, int H, int I, int E, int top_k) {
@@ -481,41 +480,6 @@ size_t moeffn_workspace_bytes(int kind, int M, int H, int I, int E, int top_k) {
   }
 }
 
-// The single-stream FFN for one or two token rows (gate/up, down and the
-// tail in one persistent kernel); *done = false when the shapes or the
-// pointers do not fit it.
-int try_ffn_stream(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, int act, const DenseWS& d, int mode,
-                   uint16_t* res, uint16_t* out, const uint16_t* norm_w, float eps, cudaStream_t s, bool* done) {
-  *done = false;
-  const int fmt = f.gate.format;
-  if (M > 2 || f.up.format != fmt || f.down.format != fmt) return MOEFFN_OK;
-  const moeffn_qweight* ws3[3] = {&f.gate, &f.up, &f.down};
-  for (const moeffn_qweight* q : ws3) {
-    if (!aligned16(q->q) || !aligned16(q->scale)) return MOEFFN_OK;
-    if (fmt == MOEFFN_Q_INT4_AFFINE_G32 && !aligned16(q->min)) return MOEFFN_OK;
-  }
-  FfnStreamArgs a{};
-  if (!ffn_stream_plan(&a, fmt, H, I, M)) return MOEFFN_OK;
-  MOEFFN_CHECK_CUDA(ffn_stream_encode(&a, fmt, to_qw(f.gate), to_qw(f.up), to_qw(f.down)), "tensor map encode");
-  a.rs_gate = static_cast<const __half*>(f.gate.scale);
-  a.rs_up = static_cast<const __half*>(f.up.scale);
-  a.rs_down = static_cast<const __half*>(f.down.scale);
-  a.act = act;
-  a.eps = eps;
-  a.x = x;
-  a.res = res;
-  a.out = out;
-  a.norm_w = norm_w;
-  a.hbuf = d.acts;
-  a.ybuf = d.d;
-  {
-    ProfScope ps("ffn_stream", s);
-    MOEFFN_CHECK_CUDA(launch_ffn_stream(a, fmt, mode, s), "single-stream FFN launch");
-  }
-  *done = true;
-  return MOEFFN_OK;
-}
-
 int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act, void* ws,
               size_t ws_bytes, moeffn_stream_t stream) {
   g_last_error.clear();
@@ -535,11 +499,6 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
   Carve cw{static_cast<char*>(ws)};
   const DenseWS d = carve_dense(cw, M, H, I);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  bool done = false;
-  if ((rc = try_ffn_stream(*w, x, M, H, I, act, d, STREAM_RESIDUAL, residual, nullptr, nullptr, 0.f, s, &done)) !=
-      MOEFFN_OK)
-    return rc;
-  if (done) return MOEFFN_OK;
   int splits = 0;
   if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits)) != MOEFFN_OK) return rc;
   TailArgs t{};
@@ -579,11 +538,6 @@ int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* no
   Carve cw{static_cast<char*>(ws)};
   const DenseWS d = carve_dense(cw, M, H, I);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  bool done = false;
-  if ((rc = try_ffn_stream(*w, x, M, H, I, act, d, STREAM_RMSNORM, nullptr, h1_out, norm_w, eps, s, &done)) !=
-      MOEFFN_OK)
-    return rc;
-  if (done) return MOEFFN_OK;
   int splits = 0;
   if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits)) != MOEFFN_OK) return rc;
   TailArgs t{};

@@ -1,5 +1,4 @@
-// Arithmetic shared by the weight-streaming GEMV kernels (gemv_tma.cu,
-// ffn_stream.cu): activations staged as int16 fixed point per weight chunk,
+// Arithmetic of the weight-streaming GEMV (gemv_tma.cu): activations staged as int16 fixed point per weight chunk,
 // codes times staged activations summed exactly in int32 with DP2A.
 #pragma once
 #include "common.cuh"

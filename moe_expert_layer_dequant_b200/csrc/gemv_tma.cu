@@ -72,9 +72,12 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   constexpr int R = NC;  // rows per stage
   extern __shared__ __align__(128) uint8_t smem[];
 
-  // No global memory access (weights included) before the previous kernel in
-  // the stream has completed: only the launch itself overlaps it.
-  pdl_wait();
+  // A dense job's producer reads only weights, which no kernel writes, so it
+  // starts streaming while the previous kernel in the stream finishes; the
+  // consumers (activations in, outputs out) and grouped jobs (whose expert
+  // lists the routing kernels write) wait for it first.
+  const bool early = a.offsets == nullptr;
+  if (!early) pdl_wait();
   if (a.stages % G != 0 || a.stages > 8) {   // ring depth the host must not choose
     if (threadIdx.x == 0) atomicOr(&g_fault_flags, 2u);
     return;
@@ -176,6 +179,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   }
 
   // ---------------- consumers ----------------
+  if (early) pdl_wait();
   const int nthreads = NC * G * 32;
   const int grp = warp / NC, wr = warp - grp * NC;  // group, row of the stage
   const uint16_t* src = job.shared ? a.x_s : a.x;

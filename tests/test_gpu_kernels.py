@@ -151,51 +151,6 @@ def test_shared_expert_small(M, shape):
     assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "h1")
 
 
-# One or two token rows whose shapes fit the single-stream FFN kernel (gate/up,
-# grid barrier, down and the tail in one launch): one and several K stages per
-# row block, row blocks spread unevenly over the CTAs, INT4 and INT8.
-STREAM_DENSE = [
-    (2, dict(H=512, I=2048)),      # INT4, one stage per row block
-    (2, dict(H=4096, I=8192)),     # INT4, two stages per row block in both phases
-    (1, dict(H=256, I=640)),       # INT8, fewer down row blocks than CTAs
-    (1, dict(H=2048, I=8256)),     # INT8, two gate/up stages; down stages of 2752 codes in two boxes
-]
-
-
-@pytest.mark.parametrize("cfg,shape", STREAM_DENSE)
-@pytest.mark.parametrize("M", [1, 2])
-def test_dense_single_stream(cfg, shape, M):
-    c = synth.scaled_config(cfg, **shape)
-    inp = synth.make_inputs(c, M, 3)
-    dl = DeviceLayer(inp)
-    lib.profile_enable(True)
-    lib.profile_read()
-    out = dl.run(inp.x, inp.residual)
-    launched = lib.profile_read()
-    lib.profile_enable(False)
-    assert list(launched) == ["ffn_stream"], launched      # one launch for the whole layer
-    assert_bf16_close(out, oracle.layer(inp), "out")
-    inp.residual = np.zeros_like(inp.residual)
-    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "h")
-    assert lib.device_faults(True) == 0
-
-
-@pytest.mark.parametrize("shape", [dict(H=1024, I=8192), dict(H=3072, I=4096)])
-@pytest.mark.parametrize("M", [1, 2])
-def test_shared_expert_single_stream(M, shape):
-    c = synth.scaled_config(3, **shape)
-    inp = synth.make_inputs(c, M, 5)
-    dl = DeviceLayer(inp)
-    lib.profile_enable(True)
-    lib.profile_read()
-    out = dl.run(inp.x, inp.residual)
-    launched = lib.profile_read()
-    lib.profile_enable(False)
-    assert list(launched) == ["ffn_stream"], launched
-    assert_bf16_close(out, oracle.layer(inp), "h1")
-    assert lib.device_faults(True) == 0
-
-
 MOE_SMALL = [
     dict(cfg=4, H=256, I=96, E=16, k=4, I_s=64),     # register-load GEMV path
     dict(cfg=5, H=320, I=192, E=8, k=2, I_s=0),
