@@ -49,6 +49,9 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--graph", action="store_true",
+                   help="time CUDA graph replays of the library calls instead of eager calls (on B200 the replays "
+                        "measured 1-3 us per step slower: the captured launches lose part of their programmatic overlap)")
     return p.parse_args()
 
 
@@ -240,6 +243,38 @@ def run_ours(args, rank, world, local_rank):
         layer.step(i, x, res, out, ws)
     torch.cuda.synchronize()
 
+    # With --graph: one CUDA graph per weight copy, each holding one step's
+    # library calls (kernel parameters, tensor maps included, fixed at
+    # capture), replayed in the timed region. Eager calls otherwise, or if a
+    # capture fails.
+    graphs = []
+    graph_error = "default; --graph replays CUDA graphs"
+    try:
+        if not args.graph:
+            raise RuntimeError("eager timing")
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            for i in range(len(layer.copies)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    layer.step(i, x, res, out, ws)
+                graphs.append(g)
+        torch.cuda.current_stream().wait_stream(cap)
+        for i in range(max(args.warmup, len(graphs))):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+    except Exception as exc:   # noqa: BLE001 - report and time eagerly
+        graphs = []
+        if args.graph:
+            graph_error = f"graph capture failed: {type(exc).__name__}: {exc}"
+
+    def timed_step(i):
+        if graphs:
+            graphs[i % len(graphs)].replay()
+        else:
+            layer.step(i, x, res, out, ws)
+
     # timed region: K steps, device events, clocks sampled meanwhile
     sampler = ClockSampler(local_rank)
     sampler.start()
@@ -249,7 +284,7 @@ def run_ours(args, rank, world, local_rank):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for i in range(args.steps):
-        layer.step(i, x, res, out, ws)
+        timed_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -340,6 +375,8 @@ def run_ours(args, rank, world, local_rank):
             "config": {
                 "workload": workload_name(c, M), "M": M, "H": c.H, "I": c.I, "format": c.fmt,
                 "act": c.act, "parallelism": "replicas" if world > 1 else "single-gpu",
+                "launch": (f"CUDA graph replay ({len(graphs)} graphs, one per weight copy, each one step of library calls)"
+                           if graphs else f"eager library calls ({graph_error})"),
                 "l2": f"weight ring of {ring} device copies; each step reads the next copy "
                       f"({per_step / 1e6:.1f} MB read per step, {ring * per_step / 1e6:.0f} MB per ring turn > 126 MB L2)",
             },
