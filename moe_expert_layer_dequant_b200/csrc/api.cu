@@ -193,12 +193,14 @@ struct Carve {
 struct DenseWS {
   uint16_t* acts;
   float* d;
+  int* cnt;   // [kSMs] arrival counters of the down projection's K splits
 };
 
 DenseWS carve_dense(Carve& c, int M, int H, int I) {
   DenseWS w;
   w.acts = c.take<uint16_t>((size_t)M * I);
   w.d = c.take<float>((size_t)down_splits_any(I) * M * H);
+  w.cnt = c.take<int>(kSMs);
   return w;
 }
 
@@ -278,9 +280,11 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 // ---- shared FFN launch (dense mode) ---------------------------------------
 
 // Gate/up + activation and the down projection (fp32 K-split partials in
-// w.d); returns the number of splits written through *splits_out.
+// w.d); returns the number of splits written through *splits_out. With `res`
+// given, a path that can also applies the residual tail (*tail_done = true).
 int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, int act, const DenseWS& w,
-                  cudaStream_t s, int* splits_out) {
+                  cudaStream_t s, int* splits_out, uint16_t* res, bool* tail_done) {
+  *tail_done = false;
   const int fmt = f.gate.format;
   if (M >= kTcMinTokens && tc_ok(f) && aligned16(x)) {
     const int mt = tc_mt_for(M), tpc = tc_tokens_per_cta(mt), tt = (M + tpc - 1) / tpc;
@@ -355,6 +359,10 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     g.ctas_per_job = kSMs;
     g.stage_tokens = gu.tokens;
     g.stages = gu.stages;
+    if (res != nullptr) {
+      g.zero_cnt = w.cnt;
+      g.zero_n = kSMs;
+    }
     {
       ProfScope ps("gateup_gemv_tma", s);
       MOEFFN_CHECK_CUDA(launch_tma_gemv(g, 2, gu.mt, 1, 1, s), "gate/up launch");
@@ -377,10 +385,15 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.ctas_per_job = std::max(1, kSMs / splits);
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;
+    if (res != nullptr) {
+      d.tile_cnt = w.cnt;
+      d.res = res;
+    }
     {
       ProfScope ps("down_gemv_tma", s);
       MOEFFN_CHECK_CUDA(launch_tma_gemv(d, 1, dn.mt, splits, 1, s), "down launch");
     }
+    *tail_done = res != nullptr;
     return MOEFFN_OK;
   }
 
@@ -500,7 +513,9 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
   const DenseWS d = carve_dense(cw, M, H, I);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int splits = 0;
-  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits)) != MOEFFN_OK) return rc;
+  bool tail_done = false;
+  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits, residual, &tail_done)) != MOEFFN_OK) return rc;
+  if (tail_done) return MOEFFN_OK;
   TailArgs t{};
   t.mode = TAIL_RESIDUAL;
   t.M = M;
@@ -539,7 +554,8 @@ int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* no
   const DenseWS d = carve_dense(cw, M, H, I);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int splits = 0;
-  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits)) != MOEFFN_OK) return rc;
+  bool tail_done = false;
+  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits, nullptr, &tail_done)) != MOEFFN_OK) return rc;
   TailArgs t{};
   t.mode = TAIL_RMSNORM;
   t.M = M;

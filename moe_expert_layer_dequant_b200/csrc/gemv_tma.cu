@@ -181,6 +181,8 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   // ---------------- consumers ----------------
   if (early) pdl_wait();
   const int nthreads = NC * G * 32;
+  if (a.zero_cnt != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    for (int i = threadIdx.x; i < a.zero_n; i += nthreads) a.zero_cnt[i] = 0;
   const int grp = warp / NC, wr = warp - grp * NC;  // group, row of the stage
   const uint16_t* src = job.shared ? a.x_s : a.x;
   const int ld = job.shared ? job.K : a.ld_x;
@@ -313,6 +315,34 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+  }
+
+  if (a.res != nullptr) {
+    // Residual tail folded in (dense down projection): the last of the K
+    // splits to finish this CTA's row range adds the splits' partial sums in
+    // split order, rounds to bf16 and adds the result to the residual, as the
+    // tail kernel would.
+    __threadfence();
+    consumer_sync(nthreads);
+    int* last = reinterpret_cast<int*>(xi);   // staged activations are no longer read
+    if (threadIdx.x == 0) {
+      const int old = atomicAdd(&a.tile_cnt[blockIdx.x], 1);
+      *last = old == (int)gridDim.y - 1;
+      if (*last) a.tile_cnt[blockIdx.x] = 0;  // ready for the next call
+    }
+    consumer_sync(nthreads);
+    if (*last) {
+      __threadfence();
+      const int nr = r1 - r0;
+      const size_t stride = (size_t)a.slots * job.N;
+      for (int i = threadIdx.x; i < nr * job.ntok; i += nthreads) {
+        const int t = i / nr, n = r0 + (i - t * nr);
+        const size_t o = (size_t)t * job.N + n;
+        float h = 0.f;
+        for (int sp = 0; sp < (int)gridDim.y; ++sp) h += __ldcg(a.out_d + sp * stride + o);
+        a.res[o] = float_to_bf16_bits(bf16_bits_to_float(a.res[o]) + round_bf16(h));
+      }
     }
   }
 }

@@ -41,6 +41,11 @@ struct TmaGemvArgs {
   uint16_t* out_act_s;         // [M][Ns]
   float* out_d;                // down: [splits][slots][N] fp32 partial sums
   float* out_d_s;              // [splits][M][N]
+  int* zero_cnt;               // gate/up, dense mode: counters cleared for the down launch that follows
+  int zero_n;
+  int* tile_cnt;               // down, dense mode: arrivals of the K splits per CTA row range
+  uint16_t* res;               // down, dense mode: residual [M][N], updated in place by the last K split
+                               // of each row range (null: fp32 partials only, a tail kernel adds them)
   int ks_len;                  // K elements per split (INT4: multiple of 256)
   int ctas_per_job;
   int stage_tokens;
