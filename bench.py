@@ -96,6 +96,23 @@ def algorithmic_flops(c: synth.LayerConfig, M: int):
     return {"gateup": gu, "down": dn}
 
 
+def max_over_ranks(dist, value: float, device) -> float:
+    """The largest of every rank's value (all ranks call this in the same
+    order); the value itself without a process group."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, M: int, steps: int, ms_total: float) -> float:
+    """Whole-job tokens/s: every rank runs M token rows per step on its own GPU
+    (replicas), timed as the slowest rank."""
+    return world * M * steps / (ms_total * 1e-3)
+
+
 def workload_name(c, M):
     return f"cfg{c.cfg} {c.name} M={M}"
 
@@ -289,11 +306,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms_total = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms_total], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(dist, e0.elapsed_time(e1), "cuda")
     ms_step = ms_total / args.steps
 
     # second pass of the same steps with per-launch events (roofline)
@@ -322,11 +335,7 @@ def run_ours(args, rank, world, local_rank):
         hout.copy_(src, non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(dist, f0.elapsed_time(f1), "cuda")
 
     # union size of the measured batch (MoE), from the library's own router
     union = None
@@ -338,7 +347,7 @@ def run_ours(args, rank, world, local_rank):
     result = None
     if rank == 0:
         hbm, bf16_tf, bf16_sus, peak_src = measured_peaks()
-        tok_s = world * M / (ms_step * 1e-3)
+        tok_s = replica_throughput(world, M, args.steps, ms_total)
         weight_gbs = ab["total"] / (ms_step * 1e-3) / 1e9
         # dominant kernel: largest share of device time in the profiled pass
         dom_name, (dom_n, dom_ms) = max(prof.items(), key=lambda kv: kv[1][1])
@@ -395,7 +404,7 @@ def run_ours(args, rank, world, local_rank):
             "kernels": {k: {"launches": n, "avg_us": round(ms / n * 1e3, 3), "share": round(ms / sum(v[1] for v in prof.values()), 4)}
                         for k, (n, ms) in prof.items()},
             "e2e": {
-                "value": round(world * M * e2e_steps / (e2e_ms * 1e-3), 2), "unit": "tokens/s",
+                "value": round(replica_throughput(world, M, e2e_steps, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(inp.x.nbytes + inp.residual.nbytes),
                 "d2h_bytes_per_step": int(inp.residual.nbytes),
             },
