@@ -309,6 +309,19 @@ def run_ours(args, rank, world, local_rank):
     ms_total = max_over_ranks(dist, e0.elapsed_time(e1), "cuda")
     ms_step = ms_total / args.steps
 
+    # per-step distribution: events around every call, in a pass of its own
+    n_dist = min(args.steps, 500)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_dist)]
+    for i in range(n_dist):
+        evs[i][0].record(stream)
+        layer.step(i, x, res, out, ws)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    st = sorted(a.elapsed_time(b) * 1000.0 for a, b in evs)
+    step_us = {"median": round(st[len(st) // 2], 3), "p10": round(st[int(0.1 * (len(st) - 1))], 3),
+               "p90": round(st[int(0.9 * (len(st) - 1))], 3), "steps": n_dist,
+               "how": "CUDA events around each call in a separate pass (value uses the uninterrupted timed loop)"}
+
     # second pass of the same steps with per-launch events (roofline)
     lib.profile_enable(True)
     lib.profile_read()
@@ -376,6 +389,7 @@ def run_ours(args, rank, world, local_rank):
             "steps": args.steps,
             "warmup": args.warmup,
             "ms_per_step": round(ms_step, 6),
+            "step_us": step_us,
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
