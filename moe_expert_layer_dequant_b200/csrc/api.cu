@@ -139,9 +139,10 @@ TmaGeom tma_geom(int fmt, int nm, int klen, int want_tokens) {
   const size_t st = tma_gemv_stage_bytes(fmt, nm, klen);
   int stages = base + 2 * st <= kTmaSmemBudget ? (int)std::min<size_t>(8, (kTmaSmemBudget - base) / st) : 0;
   // Each ring slot must belong to one consumer group (see gemv_tma.cu).
-  stages -= stages % kTmaGroups;
+  const int groups = tma_groups(fmt, nm);
+  stages -= stages % groups;
   g.stages = stages;
-  g.ok = stages >= kTmaGroups && stages >= 2;
+  g.ok = stages >= groups && stages >= 2;
   return g;
 }
 

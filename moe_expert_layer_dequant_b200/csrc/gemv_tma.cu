@@ -349,14 +349,15 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
 
 template <int FMT, int MT, int NM>
 cudaError_t launch_one(const TmaGemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-  auto kern = k_gemv_tma<FMT, MT, NM, kTmaConsumers, kTmaGroups>;
+  constexpr int G = tma_groups(FMT, NM);
+  auto kern = k_gemv_tma<FMT, MT, NM, kTmaConsumers, G>;
   static size_t smem_set = 0;  // largest dynamic shared memory opted in so far
   if (smem > smem_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     smem_set = 227 * 1024;
   }
-  return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * kTmaGroups + 1)), smem, s, a);
+  return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * G + 1)), smem, s, a);
 }
 
 template <int FMT, int NM>

@@ -7,7 +7,11 @@
 namespace moeffn {
 
 constexpr int kTmaConsumers = 8;  // consumer warps per group = rows per stage
-constexpr int kTmaGroups = 2;     // consumer groups, taking alternate stages
+// Consumer groups, taking stages in turn: three for a single INT4 matrix (the
+// down projection; more warps to hide the per-stage arithmetic latency), two
+// otherwise (the fused gate/up pair's larger stages leave room for fewer slots,
+// and the INT8 consumers need more registers than 800 threads allow).
+constexpr int tma_groups(int fmt, int nm) { return (nm == 1 && fmt == FMT_INT4_G32) ? 3 : 2; }
 
 // Tensor maps of one K-split matrix: codes (u64 elements), scales, mins (u16).
 struct QWMaps {
