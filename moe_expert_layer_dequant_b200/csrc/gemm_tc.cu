@@ -450,11 +450,6 @@ int tc_mt_for(int tokens) { return tokens > kTokRows ? 2 : 1; }
 
 int tc_tokens_per_cta(int mt) { return mt * kTokRows; }
 
-size_t tc_gemm_smem(int fmt, int mt) {
-  if (fmt == FMT_INT4_G32) return mt == 2 ? tc_smem_bytes<FMT_INT4_G32, 2>() : tc_smem_bytes<FMT_INT4_G32, 1>();
-  return mt == 2 ? tc_smem_bytes<FMT_INT8_ROW, 2>() : tc_smem_bytes<FMT_INT8_ROW, 1>();
-}
-
 cudaError_t encode_tc_weight_maps(TcMaps* m, int fmt, const QW& w, int N, int K, int box_rows) {
   cudaError_t e;
   if (fmt == FMT_INT4_G32) {

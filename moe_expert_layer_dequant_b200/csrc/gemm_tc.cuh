@@ -54,7 +54,6 @@ int tc_down_rows(int H);
 int tc_mt_for(int tokens);
 int tc_tokens_per_cta(int mt);
 
-size_t tc_gemm_smem(int fmt, int mt);
 cudaError_t encode_tc_weight_maps(TcMaps* m, int fmt, const QW& w, int N, int K, int box_rows);
 cudaError_t encode_tc_x_map(CUtensorMap* m, const uint16_t* x, int rows, int K);
 cudaError_t launch_tc_gemm(const TcGemmArgs& a, int row_tiles, int splits, int jobs, cudaStream_t s);
