@@ -366,3 +366,20 @@ def test_moe_token_rows_independent():
     full = oracle.layer(inp)
     for t in range(4):
         assert np.array_equal(oracle.layer(inp, tokens=[t])[0], full[t])
+
+
+def test_zero_gate_vector_seeds_half_the_shared_expert():
+    """w_sg = 0 and routed experts that contribute nothing: sigma(0) = 1/2, so
+    the layer output is res + bf16(bf16(shared FFN) / 2), the shared branch
+    taken from the dense FFN definition and halved exactly."""
+    c = synth.scaled_config(4, H=64, I=32, E=8, k=2, I_s=64)
+    inp = synth.make_inputs(c, 3, 4)
+    zero = FFNWeights(synth.zero_like_qweight(FMT_INT4_G32, c.I, c.H), synth.zero_like_qweight(FMT_INT4_G32, c.I, c.H),
+                      synth.zero_like_qweight(FMT_INT4_G32, c.H, c.I))
+    inp.experts = [zero] * c.E
+    inp.w_sg = np.zeros(c.H, np.uint16)
+    out = oracle.bf16_to_f64(oracle.layer(inp))
+    s = oracle.bf16(oracle.ffn_hidden(inp.shared, oracle.bf16_to_f64(inp.x), "silu"))
+    want = oracle.bf16(oracle.bf16_to_f64(inp.residual) + oracle.bf16(0.5 * s))
+    assert np.any(s != 0)
+    assert np.array_equal(out, want)
