@@ -415,12 +415,9 @@ template <int FMT, int MT, int MODE>
 cudaError_t launch_t(const TcGemmArgs& a, dim3 grid, cudaStream_t s) {
   auto kern = k_qgemm_tc<FMT, MT, MODE>;
   constexpr size_t smem = tc_smem_bytes<FMT, MT>();
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static bool opted[64] = {};
+  const cudaError_t e = opt_in_smem(kern, (int)smem, opted);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, grid, dim3(kThreads), smem, s, a);
 }
 

@@ -351,12 +351,9 @@ template <int FMT, int MT, int NM>
 cudaError_t launch_one(const TmaGemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
   constexpr int G = tma_groups(FMT, NM);
   auto kern = k_gemv_tma<FMT, MT, NM, kTmaConsumers, G>;
-  static size_t smem_set = 0;  // largest dynamic shared memory opted in so far
-  if (smem > smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-    if (e != cudaSuccess) return e;
-    smem_set = 227 * 1024;
-  }
+  static bool opted[64] = {};   // opted in to the 227 KB maximum
+  const cudaError_t e = opt_in_smem(kern, 227 * 1024, opted);
+  if (e != cudaSuccess) return e;
   return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * G + 1)), smem, s, a);
 }
 

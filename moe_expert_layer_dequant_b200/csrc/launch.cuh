@@ -4,6 +4,20 @@
 
 namespace moeffn {
 
+// Opts `kern` in to `bytes` of dynamic shared memory on the current device,
+// once per device (the attribute belongs to the device's context); `done`
+// remembers which devices have it, up to 64.
+template <typename Kernel>
+cudaError_t opt_in_smem(Kernel kern, int bytes, bool (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && done[dev]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = true;
+  return e;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                        Args&&... args) {
