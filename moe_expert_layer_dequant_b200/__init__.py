@@ -17,7 +17,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from dataclasses import dataclass
+from dataclasses import dataclass, field
 from typing import Optional, Sequence
 
 import torch
@@ -111,16 +111,30 @@ def _stream(stream) -> Optional[int]:
 
 @dataclass
 class QWeight:
-    """A quantized (or plain) matrix in device memory, W[rows][cols]."""
+    """A quantized (or plain) matrix in device memory, W[rows][cols].
+
+    The C struct handed to the library is built on the first call and reused;
+    assigning a new tensor to a field rebuilds it. Changing a tensor's storage
+    in place (``resize_``, ``set_``) after the first call is not seen: assign a
+    new tensor instead."""
     format: int
     rows: int
     cols: int
     q: torch.Tensor
     scale: Optional[torch.Tensor] = None
     min: Optional[torch.Tensor] = None
+    _cache: tuple = field(default=(None, None), init=False, repr=False, compare=False)
+
+    def _key(self) -> tuple:
+        return (self.format, self.rows, self.cols, id(self.q), id(self.scale), id(self.min))
 
     def c(self) -> _QWeight:
-        return _QWeight(self.format, self.rows, self.cols, _ptr(self.q), _ptr(self.scale), _ptr(self.min))
+        """The C struct, built once and rebuilt when a field is reassigned."""
+        key = self._key()
+        if self._cache[0] != key:
+            self._cache = (key, _QWeight(self.format, self.rows, self.cols, _ptr(self.q), _ptr(self.scale),
+                                         _ptr(self.min)))
+        return self._cache[1]
 
     @property
     def nbytes(self) -> int:
@@ -133,8 +147,14 @@ class FFN:
     up: QWeight
     down: QWeight
 
+    _cache: tuple = field(default=(None, None), init=False, repr=False, compare=False)
+
     def c(self) -> _FFN:
-        return _FFN(self.gate.c(), self.up.c(), self.down.c())
+        """The C struct, built once and rebuilt when a matrix or one of its fields changes."""
+        key = (id(self.gate), self.gate._key(), id(self.up), self.up._key(), id(self.down), self.down._key())
+        if self._cache[0] != key:
+            self._cache = (key, _FFN(self.gate.c(), self.up.c(), self.down.c()))
+        return self._cache[1]
 
     @property
     def nbytes(self) -> int:
@@ -181,9 +201,11 @@ def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
     return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device)
 
 
-def _ws(ws: Optional[torch.Tensor], need: int):
+def _ws(ws: Optional[torch.Tensor], need):
+    """(workspace, pointer, bytes); `need()` sizes one when the caller gave none
+    (a given workspace is checked by the library itself)."""
     if ws is None:
-        ws = alloc_workspace(need)
+        ws = alloc_workspace(need())
     return ws, _ptr(ws), ws.numel()
 
 
@@ -194,7 +216,7 @@ def ffn_dense(w: FFN, x: torch.Tensor, residual: torch.Tensor, act: str = "silu"
               ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """residual <- bf16(residual + bf16(FFN(x))); x, residual bf16 [M][H]."""
     M, H = x.shape
-    ws, wp, wn = _ws(ws, workspace_bytes(KIND_DENSE, M, H, w.gate.rows))
+    ws, wp, wn = _ws(ws, lambda: workspace_bytes(KIND_DENSE, M, H, w.gate.rows))
     f = w.c()
     _check(_lib.ffn_dense(ctypes.byref(f), _ptr(x), _ptr(residual), M, ACTS[act], wp, wn, _stream(stream)))
     return residual
@@ -221,7 +243,7 @@ def ffn_shared_expert(w: FFN, x: torch.Tensor, norm_w: torch.Tensor, h1_out: tor
                       eps: float = 1e-6, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """h1_out <- RMSNorm(bf16(FFN(x))) * norm_w; all bf16."""
     M, H = x.shape
-    ws, wp, wn = _ws(ws, workspace_bytes(KIND_SHARED, M, H, w.gate.rows))
+    ws, wp, wn = _ws(ws, lambda: workspace_bytes(KIND_SHARED, M, H, w.gate.rows))
     f = w.c()
     _check(_lib.ffn_shared_expert(ctypes.byref(f), _ptr(x), _ptr(norm_w), float(eps), _ptr(h1_out), M, ACTS[act],
                                   wp, wn, _stream(stream)))
@@ -234,7 +256,7 @@ def moe_router_topk(router: QWeight, x: torch.Tensor, top_k: int, logits_out=Non
     M, H = x.shape
     idx = torch.empty((M, top_k), dtype=torch.int32, device=x.device)
     w = torch.empty((M, top_k), dtype=torch.float32, device=x.device)
-    ws, wp, wn = _ws(ws, workspace_bytes(KIND_ROUTER, M, H, 0, router.rows, top_k))
+    ws, wp, wn = _ws(ws, lambda: workspace_bytes(KIND_ROUTER, M, H, 0, router.rows, top_k))
     r = router.c()
     _check(_lib.moe_router_topk(ctypes.byref(r), _ptr(x), M, top_k, _ptr(logits_out), _ptr(idx), _ptr(w),
                                 _ptr(perm), _ptr(expert_offsets), wp, wn, _stream(stream)))
@@ -280,7 +302,7 @@ def moe_layer(plan: MoePlan, x: torch.Tensor, residual: torch.Tensor, topk_idx_o
               ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """residual <- bf16(residual + bf16(seeded rank-ordered routed sum)); bf16 [M][H]."""
     M = x.shape[0]
-    ws, wp, wn = _ws(ws, plan.workspace_bytes(M))
+    ws, wp, wn = _ws(ws, lambda: plan.workspace_bytes(M))
     _check(_lib.moe_layer(plan._h, _ptr(x), _ptr(residual), M, _ptr(topk_idx_out), wp, wn, _stream(stream)))
     return residual
 
