@@ -99,6 +99,18 @@ def test_activations_match_torch():
     assert oracle.silu(np.array([64.0]))[0] == 64.0
 
 
+def test_sigmoid_matches_torch_and_gates_the_product():
+    z = torch.linspace(-40, 40, 8001, dtype=torch.float64)
+    assert np.allclose(oracle.sigmoid(z.numpy()), torch.sigmoid(z).numpy(), rtol=1e-14, atol=1e-300)
+    assert oracle.sigmoid(np.array([0.0]))[0] == 0.5
+    # bf16(silu(g) * u): act on the gate operand, one rounding to bf16 (torch's own conversion)
+    g, u = np.array([1.5, -2.0, 3.0]), np.array([2.0, 0.5, -1.0])
+    want = torch.from_numpy(g / (1.0 + np.exp(-g)) * u).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(oracle.gated_activation(g, u, "silu"), want)
+    swapped = torch.from_numpy(u / (1.0 + np.exp(-u)) * g).to(torch.bfloat16).to(torch.float64).numpy()
+    assert not np.array_equal(oracle.gated_activation(g, u, "silu"), swapped)
+
+
 # --------------------------------------------------------------------------- helpers
 
 
