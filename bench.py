@@ -4,8 +4,10 @@
 
 One step = one call of the layer (every kernel of its path) on one batch of M
 seeded synthetic token rows, with the weights resident in HBM. The default
-workload is the Llama-3-8B-shaped dense FFN (hidden 4096, intermediate 14336,
-INT4-affine group-32 weights, SiLU, raw residual add).
+workload is the Mixtral-shaped MoE prefill at M = 512 token rows (hidden 4096,
+8 experts of intermediate 14336, top-2, INT4-affine group-32 weights, SiLU, raw
+residual add), the largest configuration that fits one GPU; ``--config 2 --M 1``
+selects the Llama-3-8B-shaped dense decode step, and so on.
 
 Printed: one JSON line (rank 0) with tokens/s over all ranks, weight-stream
 GB/s, the roofline of the dominant kernel (CUDA-event durations of its launches
@@ -25,7 +27,6 @@ import statistics
 import subprocess
 import sys
 import tempfile
-import threading
 import time
 
 import numpy as np
@@ -44,8 +45,14 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--config", type=int, default=2)
-    p.add_argument("--M", type=int, default=1)
+    p.add_argument("--config", type=int, default=5)
+    p.add_argument("--M", type=int, default=512)
+    p.add_argument("--warm-seconds", type=float, default=1.0,
+                   help="after the --warmup steps, keep running back-to-back steps for at least this long so "
+                        "the GPU clocks have ramped before the timed region")
+    p.add_argument("--min-timed-seconds", type=float, default=1.5,
+                   help="the K-step timed loop is repeated until this much device time is covered (at least 3 "
+                        "repeats); value uses the median repeat, and clocks are sampled over all of them")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -220,9 +227,6 @@ class GpuLayer:
         else:
             lib.moe_layer(d["plan"], x, res, ws=ws)
 
-    def launches_per_step(self):
-        return {"dense": 3, "shared": 3, "moe": 6}[self.c.kind]
-
 
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -255,10 +259,27 @@ def run_ours(args, rank, world, local_rank):
         if dist is not None:
             dist.barrier()
 
-    # warm-up
-    for i in range(args.warmup):
-        layer.step(i, x, res, out, ws)
+    # warm-up: the --warmup steps, then back-to-back steps until at least
+    # --warm-seconds of device time have passed (a GPU starts a lease at idle
+    # clocks; a few steps are not enough for them to ramp)
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
+    n_warm = 0
+    for _ in range(args.warmup):
+        layer.step(n_warm, x, res, out, ws)
+        n_warm += 1
     torch.cuda.synchronize()
+    t_start = time.perf_counter()
+    while time.perf_counter() - t_start < args.warm_seconds:
+        for _ in range(4):
+            layer.step(n_warm, x, res, out, ws)
+            n_warm += 1
+        torch.cuda.synchronize()
+    w1.record(stream)
+    torch.cuda.synchronize()
+    est_step_ms = w0.elapsed_time(w1) / max(n_warm, 1)
+    warm_desc = (f"{args.warmup} counted steps, then back-to-back steps for >= {args.warm_seconds:g} s "
+                 f"({n_warm} steps in all)")
 
     # With --graph: one CUDA graph per weight copy, each holding one step's
     # library calls (kernel parameters, tensor maps included, fixed at
@@ -292,21 +313,29 @@ def run_ours(args, rank, world, local_rank):
         else:
             layer.step(i, x, res, out, ws)
 
-    # timed region: K steps, device events, clocks sampled meanwhile
+    # timed region: exactly K steps between events, bracketed by a barrier and
+    # a synchronize; the K-step loop is repeated (at least 3 times, until
+    # --min-timed-seconds of device time are covered) so that the clock
+    # sampler sees the GPU under load, and the median repeat is reported
+    reps = max(3, int(np.ceil(args.min_timed_seconds * 1e3 / max(est_step_ms * args.steps, 1e-3))))
+    reps = int(max_over_ranks(dist, float(min(reps, 1000)), "cuda"))   # every rank runs the same repeats
     sampler = ClockSampler(local_rank)
     sampler.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        timed_step(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    rep_ms = []
+    for _ in range(reps):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            timed_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        rep_ms.append(e0.elapsed_time(e1))
     clocks = sampler.stop()
-    ms_total = max_over_ranks(dist, e0.elapsed_time(e1), "cuda")
+    ms_total = max_over_ranks(dist, statistics.median(rep_ms), "cuda")
     ms_step = ms_total / args.steps
 
     # per-step distribution: events around every call, in a pass of its own
@@ -380,7 +409,7 @@ def run_ours(args, rank, world, local_rank):
             achieved = dom_bytes / dom_avg_s / 1e9 if dom_bytes else None
             roof_peak, roof_unit, roof_src = hbm, "GB/s", f"{peak_src} HBM copy bandwidth"
         traffic = load_traffic(c, M, dom_name)
-        launches = args.steps * sum(n for n, _ in prof.values()) // max(1, args.steps)
+        launches = sum(n for n, _ in prof.values())     # library launches of one K-step loop
         result = {
             "metric": "FFN/MoE layer tokens/s (weight-stream HBM GB/s and % of B200 roofline alongside)",
             "value": round(tok_s, 2),
@@ -393,13 +422,16 @@ def run_ours(args, rank, world, local_rank):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16" if any("gemm_tc" in k for k in prof) else "f32",
+            "dtype": dtype_label(prof, c),
             "data": "synthetic (seeded; shapes and value distributions of the configuration)",
             "config": {
                 "workload": workload_name(c, M), "M": M, "H": c.H, "I": c.I, "format": c.fmt,
                 "act": c.act, "parallelism": "replicas" if world > 1 else "single-gpu",
                 "launch": (f"CUDA graph replay ({len(graphs)} graphs, one per weight copy, each one step of library calls)"
                            if graphs else f"eager library calls ({graph_error})"),
+                "warmup": warm_desc,
+                "timing": f"median of {reps} repeats of the {args.steps}-step loop (each bracketed by a barrier and "
+                          f"a synchronize; device events)",
                 "l2": f"weight ring of {ring} device copies; each step reads the next copy "
                       f"({per_step / 1e6:.1f} MB read per step, {ring * per_step / 1e6:.0f} MB per ring turn > 126 MB L2)",
             },
@@ -430,6 +462,16 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
         dist.destroy_process_group()
     return result
+
+
+def dtype_label(prof, c):
+    """The arithmetic the path computes in, from the kernels that ran."""
+    names = list(prof)
+    wfmt = "int4-affine" if c.fmt == synth.FMT_INT4_G32 else "int8"
+    if any("gemm_tc" in k for k in names):
+        return f"bf16 ({wfmt} weights dequantized to bf16 on the tensor cores, fp32 accumulate)"
+    return (f"int16 fixed-point x {wfmt} ({wfmt} codes times activations staged as int16 with one power-of-two "
+            f"factor per 32-element chunk, exact int32 sums, fp32 scale and accumulate)")
 
 
 def load_traffic(c, M, kernel_name):

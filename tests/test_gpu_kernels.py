@@ -11,6 +11,7 @@ import torch
 import oracle
 import synth
 from conftest import read_golden
+import handbuilt
 from devutil import DeviceLayer, assert_bf16_close, dev_bf16, host_bf16, WTOL_REL
 from synth import FMT_INT4_G32, FMT_INT8_ROW
 
@@ -180,14 +181,49 @@ def test_moe_small(shape, M):
 # --------------------------------------------------------------------------- pinned edge cases
 
 
-def test_seed_is_accumulator_start_on_gpu():
-    """Hand-built layer where seeding decides the result: the GPU gives 0 exactly
-    (seed then ranks), not 2^-24 (routed sum, then shared expert)."""
-    from test_oracle import _seed_counterexample_inputs
-    li = _seed_counterexample_inputs()
+# Hand-built layers (tests/handbuilt.py, derivations in tests/golden): H = 256
+# runs the bulk-copy GEMV path, 8 replicas of the tokens (M = 8 or 16) the
+# grouped tensor-core GEMMs. Every value is exact, so the GPU must match the
+# oracle bit for bit.
+HANDBUILT_PATHS = [(256, 1), (256, 8)]
+
+
+@pytest.mark.parametrize("H,reps", HANDBUILT_PATHS)
+def test_seed_is_accumulator_start_on_gpu(H, reps):
+    """Seeding decides the result: the GPU gives 0 exactly (seed then ranks),
+    not 2^-24 (routed sum, then shared expert)."""
+    li = handbuilt.seed_counterexample(H, reps)
     dl = DeviceLayer(li)
     out = dl.run(li.x, li.residual)
-    assert oracle.bf16_to_f64(out)[0, 0] == 0.0
+    assert np.all(oracle.bf16_to_f64(out)[:, 0] == 0.0)
+    assert np.array_equal(out, oracle.layer(li))
+    dl.close()
+
+
+@pytest.mark.parametrize("H,reps", HANDBUILT_PATHS)
+def test_shared_gate_logit_sign_on_gpu(H, reps):
+    """Seeds 1.5 and 0.498046875 for gate logits +-141/128 (golden shared_gate_seed.txt)."""
+    kv, _ = read_golden("shared_gate_seed.txt")
+    li = handbuilt.shared_gate_layer(H, reps)
+    dl = DeviceLayer(li)
+    out = dl.run(li.x, li.residual)
+    want = np.tile([float(t) for t in kv["seed_feature0"]], reps)
+    assert np.array_equal(oracle.bf16_to_f64(out)[:, 0], want)
+    assert np.array_equal(out, oracle.layer(li))
+    dl.close()
+
+
+@pytest.mark.parametrize("H,reps", HANDBUILT_PATHS)
+def test_rank_weights_meet_their_own_expert_outputs_on_gpu(H, reps):
+    """y = 1 and -5 for weights (0.75, 0.25) on expert outputs 4 and -8 (golden rank_weight_pairing.txt)."""
+    kv, _ = read_golden("rank_weight_pairing.txt")
+    li = handbuilt.rank_pairing_layer(H, reps)
+    dl = DeviceLayer(li)
+    out, idx = dl.run(li.x, li.residual, topk_out=True)
+    want_idx = np.array([[int(t) for t in kv["topk_idx_token0"]], [int(t) for t in kv["topk_idx_token1"]]] * reps)
+    assert np.array_equal(idx, want_idx)
+    want = np.tile([float(t) for t in kv["y_feature0"]], reps)
+    assert np.array_equal(oracle.bf16_to_f64(out)[:, 0], want)
     assert np.array_equal(out, oracle.layer(li))
     dl.close()
 

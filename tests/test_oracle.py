@@ -16,6 +16,7 @@ import torch
 import oracle
 import synth
 from conftest import read_golden
+import handbuilt
 from synth import FFNWeights, QWeight, FMT_INT4_G32, FMT_INT8_ROW
 
 pytestmark = pytest.mark.cpu
@@ -315,41 +316,8 @@ def test_permutation_invariants():
 # --------------------------------------------------------------------------- seeded sum
 
 
-def _seed_counterexample_inputs():
-    """Hand-built layer where the seed order decides the result (exact in fp32).
-
-    H = I = 32, E = 2, k = 2, zero router (equal logits: experts 0, 1 with
-    weights 1/2, 1/2), x = e_0, shared output 2 at row 0 with w_sg = 0
-    (sigmoid = 1/2, seed = 1), expert 0 gives d = 2^-23 and expert 1 gives -2
-    at row 0, residual 0.
-    """
-    H = I = 32
-    c = synth.scaled_config(4, H=H, I=I, E=2, k=2, I_s=I)
-    z = lambda N, K: synth.zero_like_qweight(FMT_INT4_G32, N, K)   # noqa: E731
-
-    def ffn(gate00, up00, down00):
-        g, u, d = z(I, H), z(I, H), z(H, I)
-        for w, (q, s, m) in ((g, gate00), (u, up00), (d, down00)):
-            w.q[0, 0] = q
-            w.scale[0, 0] = s
-            w.min[0, 0] = m
-        return FFNWeights(g, u, d)
-
-    # gate row 0 = 64 (15*4+4) -> silu(64) = 64; up row 0 = 2^-6 -> a_0 = 1.
-    gate, up = (15, 4.0, 4.0), (1, 2.0 ** -6, 0.0)
-    shared = ffn(gate, up, (1, 2.0, 0.0))                  # s_0 = 2
-    e0 = ffn(gate, up, (2, 2.0 ** -24, 0.0))              # d_0 = 2^-23
-    e1 = ffn(gate, up, (0, 0.0, -2.0))                    # d_1 = -2
-    # min of other entries in group 0 of the gate row is 4, but x is zero there.
-    x = np.zeros((1, H), np.uint16)
-    x[0, 0] = 0x3F80
-    li = synth.LayerInputs(c, 1, 0, x, np.zeros((1, H), np.uint16), router=np.zeros((2, H), np.float32),
-                           experts=[e0, e1], shared=shared, w_sg=np.zeros(H, np.uint16))
-    return li
-
-
 def test_seed_is_accumulator_start_not_addend():
-    li = _seed_counterexample_inputs()
+    li = handbuilt.seed_counterexample()
     out, it = oracle.moe_layer(li, return_internals=True)
     assert list(it["idx"][0]) == [0, 1] and np.all(it["w"] == 0.5)
     assert it["seed"][0, 0] == 1.0
@@ -395,3 +363,36 @@ def test_zero_gate_vector_seeds_half_the_shared_expert():
     want = oracle.bf16(oracle.bf16_to_f64(inp.residual) + oracle.bf16(0.5 * s))
     assert np.any(s != 0)
     assert np.array_equal(out, want)
+
+
+def test_shared_gate_logit_sign_and_operand():
+    """The seed is bf16(s * sigmoid(w_sg . x)) with the gate logit of THIS token
+    and its sign as written (golden shared_gate_seed.txt): tokens whose logits are
+    +-141/128 get seeds 1.5 and 0.498046875; sigmoid(-logit) swaps them and a
+    zero or wrong gate vector gives 1.0 for both."""
+    kv, _ = read_golden("shared_gate_seed.txt")
+    want_logit = [float(t) for t in kv["gate_logit"]]
+    want_seed = [float(t) for t in kv["seed_feature0"]]
+    li = handbuilt.shared_gate_layer()
+    out, it = oracle.moe_layer(li, return_internals=True)
+    x = oracle.bf16_to_f64(li.x)
+    assert list(x @ oracle.bf16_to_f64(li.w_sg)) == want_logit
+    assert list(it["seed"][:, 0]) == want_seed
+    assert not np.any(it["seed"][:, 1:])
+    assert list(oracle.bf16_to_f64(out)[:, 0]) == want_seed          # residual 0, routed sum 0
+
+
+def test_rank_weights_meet_their_own_expert_outputs():
+    """Unequal routing weights (0.75, 0.25) on experts with outputs 4 and -8
+    (golden rank_weight_pairing.txt): token 0 ranks (0, 1) -> y = 1, token 1
+    ranks (1, 0) -> y = -5; weights paired with reversed ranks give -5 and 1."""
+    kv, _ = read_golden("rank_weight_pairing.txt")
+    li = handbuilt.rank_pairing_layer()
+    out, it = oracle.moe_layer(li, return_internals=True)
+    assert list(it["idx"][0]) == [int(t) for t in kv["topk_idx_token0"]]
+    assert list(it["idx"][1]) == [int(t) for t in kv["topk_idx_token1"]]
+    w = [float(t) for t in kv["weights"]]
+    assert np.array_equal(it["w"], np.array([w, w]))
+    assert it["d"][0, 0, 0] == 4.0 and it["d"][0, 1, 0] == -8.0     # rank 0 of token 0 is expert 0
+    assert it["d"][1, 0, 0] == -8.0 and it["d"][1, 1, 0] == 4.0     # rank 0 of token 1 is expert 1
+    assert list(oracle.bf16_to_f64(out)[:, 0]) == [float(t) for t in kv["y_feature0"]]
