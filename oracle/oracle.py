@@ -194,6 +194,18 @@ def rms_norm(h1: np.ndarray, w: np.ndarray, eps: float) -> np.ndarray:
     return bf16(h1 / np.sqrt(ms + eps) * w)
 
 
+def rms_norm_prologue(res_bits: np.ndarray, w_bits: np.ndarray, eps: float) -> np.ndarray:
+    """The FFN's input m = rms_norm(x, post_attention_layernorm) (bf16 bits).
+
+    [llama] module doc formula box: ``m = rms_norm(x, post_attention_layernorm)``,
+    encoded by the caller; ``encode_llama_layer_dense`` reads it from the 2-byte
+    ``moe_x`` buffer. The norm is the one the pages encode everywhere
+    (``encode_rms_norm_bf16w``, bf16 weight): reading 3, on the bf16 residual
+    row ``x``, the result rounded to bf16.
+    """
+    return bf16_bits(rms_norm(bf16_to_f64(res_bits), bf16_to_f64(w_bits), eps))
+
+
 def ffn_dense(weights, x_bits: np.ndarray, res_bits: np.ndarray, act: str) -> np.ndarray:
     """Dense llama FFN plus raw residual add; returns the new residual (bf16 bits).
 
@@ -354,6 +366,16 @@ def dense_layer(inp) -> np.ndarray:
     if c.kind == "shared":
         return ffn_shared_expert(inp.ffn, inp.x, inp.norm_w, c.act, c.eps)
     raise ValueError(c.kind)
+
+
+def layer_prenorm(inp, norm_w_bits: np.ndarray, eps: float,
+                  tokens: Optional[Sequence[int]] = None) -> np.ndarray:
+    """The layer with its input norm: m = rms_norm(residual, w), then the layer
+    on (m, residual). ``inp.x`` is not read. Dense and MoE configurations."""
+    from copy import copy
+    sub = copy(inp)
+    sub.x = rms_norm_prologue(inp.residual, norm_w_bits, eps)
+    return layer(sub, tokens=tokens)
 
 
 def layer(inp, tokens: Optional[Sequence[int]] = None) -> np.ndarray:

@@ -396,3 +396,45 @@ def test_rank_weights_meet_their_own_expert_outputs():
     assert it["d"][0, 0, 0] == 4.0 and it["d"][0, 1, 0] == -8.0     # rank 0 of token 0 is expert 0
     assert it["d"][1, 0, 0] == -8.0 and it["d"][1, 1, 0] == 4.0     # rank 0 of token 1 is expert 1
     assert list(oracle.bf16_to_f64(out)[:, 0]) == [float(t) for t in kv["y_feature0"]]
+
+
+# --------------------------------------------------------------------------- pre-FFN norm
+
+
+def test_rms_norm_prologue_golden():
+    kv, _ = read_golden("rms_norm_prologue.txt")
+    x = synth.to_bf16_bits(np.array([[float(t) for t in kv["x"]]]))
+    w = synth.to_bf16_bits(np.array([float(t) for t in kv["w"]]))
+    got = oracle.bf16_to_f64(oracle.rms_norm_prologue(x, w, float(kv["eps"][0])))[0]
+    assert list(got) == [float(t) for t in kv["expected"]]
+
+
+def test_rms_norm_prologue_closed_forms():
+    """Constant row c: m = bf16(c / sqrt(c^2 + eps) * w); eps inside the root
+    shows for small c. A row scaled by 2^k gives the same m when eps = 0."""
+    H = 64
+    w = synth.to_bf16_bits(1.0 + np.random.default_rng(8).normal(0, 0.1, H))
+    wf = oracle.bf16_to_f64(w)
+    for c, eps in ((0.5, 1e-6), (-3.0, 1e-6), (1e-3, 1e-6), (1e-3, 1e-5)):
+        x = synth.to_bf16_bits(np.full((1, H), c))
+        cf = oracle.bf16_to_f64(x)[0, 0]
+        want = oracle.bf16(cf / math.sqrt(cf * cf + eps) * wf)
+        assert np.array_equal(oracle.bf16_to_f64(oracle.rms_norm_prologue(x, w, eps))[0], want)
+    x = synth.to_bf16_bits(np.random.default_rng(9).standard_normal((3, H)))
+    x8 = synth.to_bf16_bits(oracle.bf16_to_f64(x) * 8.0)
+    assert np.array_equal(oracle.rms_norm_prologue(x, w, 0.0), oracle.rms_norm_prologue(x8, w, 0.0))
+
+
+def test_prenorm_layer_feeds_the_normed_residual():
+    """layer_prenorm = the layer on x = rms_norm(residual), residual added raw;
+    it reads the residual twice (norm input, then the add) and never inp.x."""
+    c = synth.scaled_config(2, H=64, I=96)
+    inp = synth.make_inputs(c, 2, 3)
+    w = synth.to_bf16_bits(1.0 + np.random.default_rng(1).normal(0, 0.1, c.H))
+    got = oracle.layer_prenorm(inp, w, 1e-6)
+    inp2 = synth.make_inputs(c, 2, 3)
+    inp2.x = np.zeros_like(inp2.x) + np.uint16(0x3F80)        # a different x changes nothing
+    assert np.array_equal(oracle.layer_prenorm(inp2, w, 1e-6), got)
+    m = oracle.rms_norm_prologue(inp.residual, w, 1e-6)
+    want = oracle.ffn_dense(inp.ffn, m, inp.residual, "silu")
+    assert np.array_equal(got, want)
