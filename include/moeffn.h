@@ -117,6 +117,20 @@ const char* moeffn_last_error(void);
 int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act,
               void* ws, size_t ws_bytes, moeffn_stream_t stream);
 
+/* ffn_dense with the layer's input norm folded in:
+ *   m = bf16(x / sqrt(mean(x^2) + eps) * norm_w)   (fp32, over the H columns)
+ *   residual[t] = bf16(residual[t] + bf16(down(bf16(act(gate m_t) * (up m_t)))))
+ * with x = residual (read before it is updated). turbospark-runtime 0.3.0,
+ * src/families/llama/dense.rs, module doc formula box
+ * ("m = rms_norm(x, post_attention_layernorm)", there encoded by the caller)
+ * and encode_llama_layer_dense; the norm is the one the pages encode as
+ * encode_rms_norm_bf16w. norm_w: [H] bf16, 16-byte aligned; eps >= 0.
+ * Few token rows: the norm runs inside the gate/up kernel's staging of the
+ * token rows (no launch of its own); more rows: one small launch writes m into
+ * the workspace first. Workspace and errors as ffn_dense. */
+int ffn_dense_prenorm(const moeffn_ffn* w, const uint16_t* norm_w, float eps, uint16_t* residual, int M,
+                      int act, void* ws, size_t ws_bytes, moeffn_stream_t stream);
+
 /* Dense FFN plus residual add without a caller workspace. No counterpart on
  * the pages. For callers that cannot allocate device memory at the point of
  * the call: code inside a stream capture that must not add allocations,
@@ -167,7 +181,23 @@ typedef struct moeffn_moe_desc {
   moeffn_qweight router;              /* F32 or BF16 [E][H] */
   const moeffn_ffn* experts;          /* host array [E]; INT4-affine only */
   const moeffn_ffn* shared;           /* NULL: no shared expert (routed sum starts at 0) */
-  const moeffn_qweight* shared_gate;  /* BF16 [1][H]; required with `shared` */
+  const moeffn_qweight* shared_gate;  /* BF16 [1][H]; required with `shared` in the Qwen form */
+  /* Gemma form of the routed layer (turbospark-runtime 0.3.0,
+   * src/families/qwen/moe_batch.rs, module doc: Gemma's routed sum starts
+   * from nothing, its shared branch joins in the tail after a norm, and
+   * router_topk_gemma4 takes a learned per-expert scale;
+   * turbospark-runtime 0.1.0, src/families/gemma4/shared_expert.rs: the
+   * shared branch is the FFN then post_feedforward_layernorm_1). Appended
+   * fields; all zero for the Qwen form. */
+  const float* expert_scale;          /* device fp32 [E]: routing weight of expert e is
+                                         fp16(softmax * expert_scale[e]); NULL: ones */
+  const uint16_t* shared_post_norm;   /* device bf16 [H], 16-byte aligned: the shared expert is not
+                                         gated and does not seed the sum; its output s becomes
+                                         h1 = bf16(s / sqrt(mean(s^2) + eps) * w) and the tail is
+                                         residual = bf16(residual + bf16(y + h1)), y the routed sum
+                                         from 0. Requires `shared`, forbids `shared_gate`. NULL:
+                                         the Qwen form. */
+  float shared_post_norm_eps;         /* eps of that norm (the pages: 1e-6) */
 } moeffn_moe_desc;
 
 typedef struct moeffn_moe_plan moeffn_moe_plan;
@@ -182,12 +212,22 @@ size_t moe_workspace_bytes(const moeffn_moe_plan* plan, int M);
  *   y[t] = bf16( ((seed[t] + w_0 d_0) + w_1 d_1) + ... )  (fp32, rank order)
  *   residual[t] = bf16(residual[t] + y[t])
  * seed = bf16(bf16(shared(x_t)) * sigmoid(shared_gate . x_t)), or 0.
+ * Gemma form (shared_post_norm given): seed = 0 and
+ *   residual[t] = bf16(residual[t] + bf16(y[t] + h1[t])), h1 the normed shared branch.
  * turbospark-runtime 0.3.0, src/families/qwen/moe_batch.rs, module doc ("this
  * family's phase 2 SEEDS its accumulator with the gated shared-expert output",
  * "NO SANDWICH NORMS") and encode_qwen_layer_moe_batched.
  * topk_idx_out: optional [M][k] int32 copy of the selected experts. */
 int moe_layer(moeffn_moe_plan* plan, const uint16_t* x, uint16_t* residual, int M, int32_t* topk_idx_out,
               void* ws, size_t ws_bytes, moeffn_stream_t stream);
+
+/* moe_layer with the layer's input norm folded in: the router kernel forms
+ * m = bf16(x / sqrt(mean(x^2) + eps) * norm_w) from x = residual, uses it for
+ * the logits (and the shared-expert gate) and stores it in the workspace for
+ * the expert and shared-expert projections; then as moe_layer. Sources as
+ * ffn_dense_prenorm and moe_layer. norm_w: [H] bf16, 16-byte aligned. */
+int moe_layer_prenorm(moeffn_moe_plan* plan, const uint16_t* norm_w, float eps, uint16_t* residual, int M,
+                      int32_t* topk_idx_out, void* ws, size_t ws_bytes, moeffn_stream_t stream);
 
 /* Failure detection. Pipeline waits inside the kernels are bounded (about one
  * second); a wait that runs out sets a bit in a device fault word and the
@@ -221,6 +261,21 @@ int moeffn_test_dequant(const moeffn_qweight* w, float* out_f32, uint16_t* out_b
 int moeffn_test_topk_from_logits(const float* logits, int M, int E, int top_k, int32_t* topk_idx,
                                  float* topk_w, int32_t* perm, int32_t* expert_offsets,
                                  int32_t* union_out, int32_t* n_union_out, moeffn_stream_t stream);
+
+/* Failure injection for tests of the failure detection above (no counterpart
+ * on the pages). One-shot: applies to the next ffn_dense / ffn_shared_expert
+ * call whose gate/up projection runs the weight-streaming GEMV, then clears.
+ *  kind 1: that launch's producer issues no weight stage from stage `value`
+ *          on, as if it had died; the consumers' bounded waits run out after
+ *          `wait_us` microseconds, set bit 0 of the fault word and the kernel
+ *          finishes without its result (no copy is left in flight).
+ *  kind 2: that launch gets ring depth `value` (1..8); a depth the kernel
+ *          cannot use (not a multiple of its consumer group count) is refused
+ *          by the kernel, which sets bit 1 and returns at once.
+ *  kind 0: cancel a pending injection.
+ * wait_us: 1..1000000. The call's outputs are garbage; the next call is not
+ * affected. Returns MOEFFN_ERR_INVALID for other arguments. Not thread-safe. */
+int moeffn_test_inject_gemv_fault(int kind, int value, unsigned int wait_us);
 
 #ifdef __cplusplus
 }

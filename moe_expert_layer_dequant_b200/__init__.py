@@ -9,6 +9,8 @@ names of the C ABI (include/moeffn.h):
 * ``moe_router_topk``    -- router GEMV, top-k softmax, grouped pair order
 * ``MoePlan`` / ``moe_layer`` -- routed MoE layer with a seeded rank-ordered
   sum and a raw residual add (in place)
+* ``ffn_dense_prenorm`` / ``moe_layer_prenorm`` -- the same layers with their
+  input RMSNorm (m = rms_norm(residual, w)) applied inside the library
 
 There is no CPU fallback: importing this package fails if the library is
 missing, and every call raises ``MoeffnError`` on a non-zero status.
@@ -58,7 +60,8 @@ class _FFN(ctypes.Structure):
 class _MoeDesc(ctypes.Structure):
     _fields_ = [("num_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("act", ctypes.c_int32),
                 ("router", _QWeight), ("experts", ctypes.POINTER(_FFN)), ("shared", ctypes.POINTER(_FFN)),
-                ("shared_gate", ctypes.POINTER(_QWeight))]
+                ("shared_gate", ctypes.POINTER(_QWeight)), ("expert_scale", ctypes.c_void_p),
+                ("shared_post_norm", ctypes.c_void_p), ("shared_post_norm_eps", ctypes.c_float)]
 
 
 _vp, _sz, _i, _f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
@@ -67,6 +70,8 @@ _SIGS = {
     "moeffn_last_error": (ctypes.c_char_p, []),
     "ffn_dense": (_i, [ctypes.POINTER(_FFN), _vp, _vp, _i, _i, _vp, _sz, _vp]),
     "ffn_dense_noalloc": (_i, [ctypes.POINTER(_FFN), _vp, _vp, _i, _i, _vp]),
+    "ffn_dense_prenorm": (_i, [ctypes.POINTER(_FFN), _vp, _f, _vp, _i, _i, _vp, _sz, _vp]),
+    "moe_layer_prenorm": (_i, [_vp, _vp, _f, _vp, _i, _vp, _vp, _sz, _vp]),
     "ffn_shared_expert": (_i, [ctypes.POINTER(_FFN), _vp, _vp, _f, _vp, _i, _i, _vp, _sz, _vp]),
     "moe_router_topk": (_i, [ctypes.POINTER(_QWeight), _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_plan_create": (_i, [ctypes.POINTER(_MoeDesc), ctypes.POINTER(_vp)]),
@@ -78,6 +83,7 @@ _SIGS = {
     "moeffn_device_faults": (ctypes.c_uint, [_i]),
     "moeffn_profile_read": (_i, [ctypes.c_char_p, _i, _vp, _vp, _i, ctypes.POINTER(_i)]),
     "moeffn_test_topk_from_logits": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moeffn_test_inject_gemv_fault": (_i, [_i, _i, ctypes.c_uint]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -113,10 +119,10 @@ def _stream(stream) -> Optional[int]:
 class QWeight:
     """A quantized (or plain) matrix in device memory, W[rows][cols].
 
-    The C struct handed to the library is built on the first call and reused;
-    assigning a new tensor to a field rebuilds it. Changing a tensor's storage
-    in place (``resize_``, ``set_``) after the first call is not seen: assign a
-    new tensor instead."""
+    The C struct handed to the library is built on the first call and reused
+    while every field's device pointer and element count stay the same; a new
+    tensor in a field, or a tensor whose storage moved (``set_``, ``resize_``),
+    rebuilds it."""
     format: int
     rows: int
     cols: int
@@ -126,7 +132,9 @@ class QWeight:
     _cache: tuple = field(default=(None, None), init=False, repr=False, compare=False)
 
     def _key(self) -> tuple:
-        return (self.format, self.rows, self.cols, id(self.q), id(self.scale), id(self.min))
+        def k(t):
+            return None if t is None else (t.data_ptr(), t.numel())
+        return (self.format, self.rows, self.cols, k(self.q), k(self.scale), k(self.min))
 
     def c(self) -> _QWeight:
         """The C struct, built once and rebuilt when a field is reassigned."""
@@ -151,7 +159,7 @@ class FFN:
 
     def c(self) -> _FFN:
         """The C struct, built once and rebuilt when a matrix or one of its fields changes."""
-        key = (id(self.gate), self.gate._key(), id(self.up), self.up._key(), id(self.down), self.down._key())
+        key = (self.gate._key(), self.up._key(), self.down._key())
         if self._cache[0] != key:
             self._cache = (key, _FFN(self.gate.c(), self.up.c(), self.down.c()))
         return self._cache[1]
@@ -222,6 +230,17 @@ def ffn_dense(w: FFN, x: torch.Tensor, residual: torch.Tensor, act: str = "silu"
     return residual
 
 
+def ffn_dense_prenorm(w: FFN, norm_w: torch.Tensor, residual: torch.Tensor, act: str = "silu", eps: float = 1e-6,
+                      ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """residual <- bf16(residual + bf16(FFN(rms_norm(residual, norm_w)))); the input norm runs in the library."""
+    M, H = residual.shape
+    ws, wp, wn = _ws(ws, lambda: workspace_bytes(KIND_DENSE, M, H, w.gate.rows))
+    f = w.c()
+    _check(_lib.ffn_dense_prenorm(ctypes.byref(f), _ptr(norm_w), float(eps), _ptr(residual), M, ACTS[act], wp, wn,
+                                  _stream(stream)))
+    return residual
+
+
 NOALLOC_SCRATCH_BYTES = 4 << 20
 
 
@@ -264,20 +283,32 @@ def moe_router_topk(router: QWeight, x: torch.Tensor, top_k: int, logits_out=Non
 
 
 class MoePlan:
-    """A routed MoE layer: router, E expert FFNs (INT4-affine), optional gated shared expert."""
+    """A routed MoE layer: router, E expert FFNs (INT4-affine), optional shared expert.
+
+    Qwen form (default): the shared expert is gated by sigmoid(shared_gate . x)
+    and seeds the routed sum. Gemma form (``shared_post_norm`` given): the
+    shared branch is normed (post-FFN RMSNorm, ``shared_post_norm_eps``) and
+    joins in the tail; ``expert_scale`` (fp32 [E]) scales the routing weights.
+    """
 
     def __init__(self, router: QWeight, experts: Sequence[FFN], top_k: int, act: str = "silu",
-                 shared: Optional[FFN] = None, shared_gate: Optional[QWeight] = None):
+                 shared: Optional[FFN] = None, shared_gate: Optional[QWeight] = None,
+                 expert_scale: Optional[torch.Tensor] = None, shared_post_norm: Optional[torch.Tensor] = None,
+                 shared_post_norm_eps: float = 1e-6):
         self.router, self.experts, self.shared, self.shared_gate = router, list(experts), shared, shared_gate
+        self.expert_scale, self.shared_post_norm = expert_scale, shared_post_norm
         self.top_k, self.E, self.H = top_k, len(experts), router.cols
         arr = (_FFN * len(experts))(*[e.c() for e in experts])
         self._keep = [arr]
-        desc = _MoeDesc(len(experts), top_k, ACTS[act], router.c(), arr, None, None)
+        desc = _MoeDesc(len(experts), top_k, ACTS[act], router.c(), arr, None, None,
+                        _ptr(expert_scale), _ptr(shared_post_norm), float(shared_post_norm_eps))
         if shared is not None:
             sf = _FFN(shared.gate.c(), shared.up.c(), shared.down.c())
-            sg = shared_gate.c()
-            self._keep += [sf, sg]
+            self._keep.append(sf)
             desc.shared = ctypes.pointer(sf)
+        if shared_gate is not None:
+            sg = shared_gate.c()
+            self._keep.append(sg)
             desc.shared_gate = ctypes.pointer(sg)
         h = ctypes.c_void_p()
         _check(_lib.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)))
@@ -304,6 +335,17 @@ def moe_layer(plan: MoePlan, x: torch.Tensor, residual: torch.Tensor, topk_idx_o
     M = x.shape[0]
     ws, wp, wn = _ws(ws, lambda: plan.workspace_bytes(M))
     _check(_lib.moe_layer(plan._h, _ptr(x), _ptr(residual), M, _ptr(topk_idx_out), wp, wn, _stream(stream)))
+    return residual
+
+
+def moe_layer_prenorm(plan: MoePlan, norm_w: torch.Tensor, residual: torch.Tensor, eps: float = 1e-6,
+                      topk_idx_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """moe_layer on m = rms_norm(residual, norm_w), formed inside the library."""
+    M = residual.shape[0]
+    ws, wp, wn = _ws(ws, lambda: plan.workspace_bytes(M))
+    _check(_lib.moe_layer_prenorm(plan._h, _ptr(norm_w), float(eps), _ptr(residual), M, _ptr(topk_idx_out), wp, wn,
+                                  _stream(stream)))
     return residual
 
 
@@ -339,6 +381,14 @@ def test_dequant(w: QWeight, want_f32=True, want_bf16=True, stream=None):
     return f, b
 
 
+def test_inject_gemv_fault(kind: int, value: int = 0, wait_us: int = 2000) -> None:
+    """One-shot failure injection into the next dense gate/up GEMV launch (test export):
+    kind 1 stops its producer at stage `value` (bounded waits of `wait_us` run out,
+    fault bit 0), kind 2 forces ring depth `value` (refused by the kernel, fault bit 1),
+    kind 0 cancels."""
+    _check(_lib.moeffn_test_inject_gemv_fault(kind, value, wait_us))
+
+
 def test_topk_from_logits(logits: torch.Tensor, top_k: int, stream=None):
     """Top-k / weights / grouped order from given fp32 logits (test export)."""
     M, E = logits.shape
@@ -354,6 +404,6 @@ def test_topk_from_logits(logits: torch.Tensor, top_k: int, stream=None):
     return idx, w, perm, offs, uni[: int(nu.item())]
 
 
-__all__ = ["ffn_dense", "ffn_dense_noalloc", "ffn_shared_expert", "moe_router_topk", "moe_layer", "MoePlan", "QWeight", "FFN",
+__all__ = ["ffn_dense", "ffn_dense_prenorm", "moe_layer_prenorm", "ffn_dense_noalloc", "ffn_shared_expert", "moe_router_topk", "moe_layer", "MoePlan", "QWeight", "FFN",
            "qweight_from_arrays", "upload_qweight", "upload_ffn", "plain_weight", "workspace_bytes", "alloc_workspace", "test_dequant",
-           "test_topk_from_logits", "profile_enable", "profile_read", "device_faults", "MoeffnError", "LIB_PATH"]
+           "test_topk_from_logits", "test_inject_gemv_fault", "profile_enable", "profile_read", "device_faults", "MoeffnError", "LIB_PATH"]

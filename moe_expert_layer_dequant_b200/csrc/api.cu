@@ -22,6 +22,15 @@ namespace {
 
 thread_local std::string g_last_error;
 
+// One-shot failure injection for the next dense gate/up GEMV launch
+// (moeffn_test_inject_gemv_fault; failure-detection tests only).
+struct GemvInjection {
+  int kind = 0;                      // 0 none, 1 producer stops, 2 ring depth
+  int value = 0;
+  unsigned long long wait_ns = 0;
+};
+GemvInjection g_inject;
+
 int fail(int code, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -132,7 +141,7 @@ struct TmaGeom {
 TmaGeom tma_geom(int fmt, int nm, int klen, int want_tokens) {
   TmaGeom g{};
   g.mt = want_tokens <= 1 ? 1 : 2;
-  const size_t per_tok = tma_gemv_smem(fmt, nm, klen, 1, 1, 0) - 128;
+  const size_t per_tok = tma_gemv_smem(fmt, nm, klen, 1, 1, 0) - tma_gemv_smem(fmt, nm, klen, 0, 1, 0);
   int t = (int)std::max<size_t>(1, kTmaXBudget / std::max<size_t>(per_tok, 1));
   g.tokens = std::max(1, std::min(want_tokens, t));
   const size_t base = tma_gemv_smem(fmt, nm, klen, g.tokens, g.mt, 0);
@@ -159,10 +168,10 @@ int mt_for(int tokens) { return tokens <= 1 ? 1 : 2; }
 constexpr int kTcMinTokens = 6;      // dense: token rows from which the GEMM replaces the GEMV
 constexpr int kTcMinMoeTokens = 8;   // MoE layer: token rows from which the grouped GEMMs are used
 
-// Rows a multiple of 16 keep every 8-column output chunk of the epilogue
-// inside the matrix and 16-byte aligned.
+// The GEMM's weight stages cover 256 (INT4) or 128 (INT8) K elements, loaded
+// by TMA from 16-byte aligned rows.
 bool tc_ok(const moeffn_qweight& w) {
-  if (!aligned16(w.q) || w.rows % 16 != 0) return false;
+  if (!aligned16(w.q)) return false;
   if (w.format == MOEFFN_Q_INT4_AFFINE_G32) return w.cols % 256 == 0 && aligned16(w.scale) && aligned16(w.min);
   return w.format == MOEFFN_Q_INT8_ROW && w.cols % 128 == 0 && aligned16(w.scale);
 }
@@ -195,6 +204,7 @@ struct DenseWS {
   uint16_t* acts;
   float* d;
   int* cnt;   // [kSMs] arrival counters of the down projection's K splits
+  uint16_t* m;   // [M][H] the normed input, when the layer applies its input norm
 };
 
 DenseWS carve_dense(Carve& c, int M, int H, int I) {
@@ -202,6 +212,7 @@ DenseWS carve_dense(Carve& c, int M, int H, int I) {
   w.acts = c.take<uint16_t>((size_t)M * I);
   w.d = c.take<float>((size_t)down_splits_any(I) * M * H);
   w.cnt = c.take<int>(kSMs);
+  w.m = c.take<uint16_t>((size_t)M * H);
   return w;
 }
 
@@ -220,6 +231,7 @@ struct MoeWS {
   float* d;
   float* d_s;
   uint16_t* xg;      // token rows in pair-slot order (grouped GEMM operand)
+  uint16_t* m;       // [M][H] the normed input, when the layer applies its input norm
 };
 
 // Down-projection K split shared by the routed and the shared expert jobs.
@@ -253,6 +265,7 @@ MoeWS carve_moe(Carve& c, int M, int H, int Ie, int Is, int E, int k) {
   w.d = c.take<float>((size_t)sp.routed * P * H);
   w.d_s = c.take<float>((size_t)sp.shared * M * H);
   w.xg = c.take<uint16_t>(P * H);
+  w.m = c.take<uint16_t>((size_t)M * H);
   return w;
 }
 
@@ -280,22 +293,38 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 // ---- shared FFN launch (dense mode) ---------------------------------------
 
+// The layer's input m = rms_norm(x, norm_w) into w.m (one launch).
+int launch_prenorm(const uint16_t* x, const uint16_t* norm_w, float eps, int M, int H, const DenseWS& w,
+                   cudaStream_t s) {
+  PrenormArgs pa{x, norm_w, eps, M, H, w.m};
+  ProfScope ps("prenorm_rows", s);
+  MOEFFN_CHECK_CUDA(launch_prenorm_rows(pa, s), "input norm launch");
+  return MOEFFN_OK;
+}
+
 // Gate/up + activation and the down projection (fp32 K-split partials in
 // w.d); returns the number of splits written through *splits_out. With `res`
 // given, a path that can also applies the residual tail (*tail_done = true).
+// With `norm_w`, x is the un-normed residual and the layer's input is
+// m = rms_norm(x, norm_w): folded into the GEMV's activation staging, or
+// written to w.m by a launch of its own before the GEMMs.
 int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, int act, const DenseWS& w,
-                  cudaStream_t s, int* splits_out, uint16_t* res, bool* tail_done) {
+                  cudaStream_t s, int* splits_out, uint16_t* res, bool* tail_done, const uint16_t* norm_w = nullptr,
+                  float eps = 0.f) {
   *tail_done = false;
   const int fmt = f.gate.format;
+  int rc;
   if (M >= kTcMinTokens && tc_ok(f) && aligned16(x)) {
-    const int mt = tc_mt_for(M), tpc = tc_tokens_per_cta(mt), tt = (M + tpc - 1) / tpc;
-    const int fg = tc_gateup_feat(I), rd = tc_down_rows(H);
+    if (norm_w != nullptr) {
+      if ((rc = launch_prenorm(x, norm_w, eps, M, H, w, s)) != MOEFFN_OK) return rc;
+      x = w.m;
+    }
+    const int ntile = tc_ntile_for(M), tt = (M + ntile - 1) / ntile;
     TcGemmArgs g{};
     g.fmt = fmt;
     g.act = act;
     g.mode = TC_GATEUP;
-    g.mt = mt;
-    g.tile = fg;
+    g.ntile = ntile;
     g.N = I;
     g.K = H;
     g.M = M;
@@ -305,18 +334,17 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     g.token_tiles = tt;
     g.rscale0 = static_cast<const __half*>(f.gate.scale);
     g.rscale1 = static_cast<const __half*>(f.up.scale);
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, x, M, H), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w0, fmt, to_qw(f.gate), I, H, fg), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w1, fmt, to_qw(f.up), I, H, fg), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, x, M, H, ntile), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w0, fmt, to_qw(f.gate), I, H), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&g.w1, fmt, to_qw(f.up), I, H), "tensor map encode");
     {
       ProfScope ps("gateup_gemm_tc", s);
-      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (I + fg - 1) / fg, 1, 1, s), "gate/up GEMM launch");
+      MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (I + kTcGateUpFeat - 1) / kTcGateUpFeat, 1, 1, s), "gate/up GEMM launch");
     }
     TcGemmArgs d{};
     d.fmt = fmt;
     d.mode = TC_DOWN;
-    d.mt = mt;
-    d.tile = rd;
+    d.ntile = ntile;
     d.N = H;
     d.K = I;
     d.M = M;
@@ -324,12 +352,12 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.out_d = w.d;
     d.token_tiles = tt;
     d.rscale0 = static_cast<const __half*>(f.down.scale);
-    const int row_tiles = (H + rd - 1) / rd;
+    const int row_tiles = (H + kTcDownRows - 1) / kTcDownRows;
     const int want = (kSMs + row_tiles * tt - 1) / (row_tiles * tt);
     d.ks_len = tc_down_slice(I, fmt, want, down_splits_any(I));
     const int splits = (I + d.ks_len - 1) / d.ks_len;
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, M, I), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&d.w0, fmt, to_qw(f.down), H, I, rd), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, M, I, ntile), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&d.w0, fmt, to_qw(f.down), H, I), "tensor map encode");
     {
       ProfScope ps("down_gemm_tc", s);
       MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, splits, 1, s), "down GEMM launch");
@@ -363,6 +391,21 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     if (res != nullptr) {
       g.zero_cnt = w.cnt;
       g.zero_n = kSMs;
+    }
+    if (norm_w != nullptr) {
+      if (gu.tokens <= 8) {            // folded into the staging of the token rows
+        g.norm_w = norm_w;
+        g.eps = eps;
+      } else {
+        if ((rc = launch_prenorm(x, norm_w, eps, M, H, w, s)) != MOEFFN_OK) return rc;
+        g.x = w.m;
+      }
+    }
+    if (g_inject.kind != 0) {          // failure-detection tests only
+      if (g_inject.kind == 1) g.inject_stop = g_inject.value + 1;
+      if (g_inject.kind == 2) g.stages = g_inject.value;
+      g.wait_ns = g_inject.wait_ns;
+      g_inject = GemvInjection{};
     }
     {
       ProfScope ps("gateup_gemv_tma", s);
@@ -398,6 +441,10 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     return MOEFFN_OK;
   }
 
+  if (norm_w != nullptr) {
+    if ((rc = launch_prenorm(x, norm_w, eps, M, H, w, s)) != MOEFFN_OK) return rc;
+    x = w.m;
+  }
   GateUpArgs g{};
   g.fmt = fmt;
   g.act = act;
@@ -449,6 +496,9 @@ struct moeffn_moe_plan {
   const uint16_t* w_sg;
   moeffn_ffn shared;
   bool has_shared;
+  const float* expert_scale = nullptr;         // per-expert routing scale (null: ones)
+  const uint16_t* shared_post_norm = nullptr;  // Gemma form: the shared branch's post-FFN norm weight
+  float shared_post_norm_eps = 0.f;
   bool tma;               // every expert (and the shared one) fits the TMA GEMV
   QW* d_gate = nullptr;   // device tables [E]
   QW* d_up = nullptr;
@@ -456,16 +506,30 @@ struct moeffn_moe_plan {
   QWMaps* d_maps = nullptr;    // [E] tensor maps of the expert down matrices (K split)
   QWMaps* d_maps_s = nullptr;  // [1] shared expert down (K split)
   bool tc = false;             // tensor-core GEMM maps built
-  TcMaps* d_tc_gate = nullptr; // [E] (boxes of tc_fe rows)
-  TcMaps* d_tc_up = nullptr;   // [E] (boxes of tc_fe rows)
-  TcMaps* d_tc_down = nullptr; // [E] (boxes of tc_rd rows)
-  TcMaps tc_sg{}, tc_su{}, tc_sd{};   // shared expert (tc_fs, tc_fs, tc_rd rows)
-  int tc_fe = 0, tc_fs = 0, tc_rd = 0; // GATEUP features per tile (routed, shared), DOWN rows per tile
+  TcMaps* d_tc_gate = nullptr; // [E]
+  TcMaps* d_tc_up = nullptr;   // [E]
+  TcMaps* d_tc_down = nullptr; // [E]
+  TcMaps tc_sg{}, tc_su{}, tc_sd{};   // shared expert
 };
 
 extern "C" {
 
 const char* moeffn_last_error(void) { return g_last_error.c_str(); }
+
+int moeffn_test_inject_gemv_fault(int kind, int value, unsigned int wait_us) {
+  g_last_error.clear();
+  if (kind == 0) {
+    g_inject = GemvInjection{};
+    return MOEFFN_OK;
+  }
+  if ((kind != 1 && kind != 2) || value < 0 || (kind == 2 && (value < 1 || value > 8)) || wait_us == 0 ||
+      wait_us > 1000000u)
+    return fail(MOEFFN_ERR_INVALID, "moeffn_test_inject_gemv_fault: kind %d value %d wait %u us", kind, value, wait_us);
+  g_inject.kind = kind;
+  g_inject.value = value;
+  g_inject.wait_ns = 1000ull * wait_us;
+  return MOEFFN_OK;
+}
 
 unsigned int moeffn_device_faults(int clear) {
   // Blocking read of the kernels' fault words (bounded waits that ran out).
@@ -494,19 +558,29 @@ size_t moeffn_workspace_bytes(int kind, int M, int H, int I, int E, int top_k) {
   }
 }
 
-int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act, void* ws,
-              size_t ws_bytes, moeffn_stream_t stream) {
+namespace {
+
+// ffn_dense and ffn_dense_prenorm: with norm_w, x is null and the input is
+// m = rms_norm(residual, norm_w).
+int dense_entry(const char* who, const moeffn_ffn* w, const uint16_t* x, const uint16_t* norm_w, float eps,
+                uint16_t* residual, int M, int act, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
   g_last_error.clear();
-  if (w == nullptr || x == nullptr || residual == nullptr) return fail(MOEFFN_ERR_INVALID, "ffn_dense: null pointer");
-  if (M < 1) return fail(MOEFFN_ERR_INVALID, "ffn_dense: M=%d", M);
-  if (act != MOEFFN_ACT_SILU && act != MOEFFN_ACT_GELU_TANH) return fail(MOEFFN_ERR_INVALID, "ffn_dense: act=%d", act);
+  if (w == nullptr || residual == nullptr || (x == nullptr && norm_w == nullptr))
+    return fail(MOEFFN_ERR_INVALID, "%s: null pointer", who);
+  if (M < 1) return fail(MOEFFN_ERR_INVALID, "%s: M=%d", who, M);
+  if (act != MOEFFN_ACT_SILU && act != MOEFFN_ACT_GELU_TANH) return fail(MOEFFN_ERR_INVALID, "%s: act=%d", who, act);
   const int H = w->gate.cols, I = w->gate.rows;
-  int rc = check_ffn(*w, "ffn_dense", H, I);
+  int rc = check_ffn(*w, who, H, I);
   if (rc != MOEFFN_OK) return rc;
-  if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "ffn_dense: x/residual not 16-byte aligned");
-  if (x == residual) return fail(MOEFFN_ERR_INVALID, "ffn_dense: x aliases residual");
+  if (norm_w != nullptr) {
+    if (!aligned16(norm_w)) return fail(MOEFFN_ERR_INVALID, "%s: norm weight not 16-byte aligned", who);
+    if (!(eps >= 0.0f)) return fail(MOEFFN_ERR_INVALID, "%s: eps must be >= 0", who);
+    x = residual;
+  }
+  if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "%s: x/residual not 16-byte aligned", who);
+  if (norm_w == nullptr && x == residual) return fail(MOEFFN_ERR_INVALID, "%s: x aliases residual", who);
   if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax || gemv_stage_bytes(w->gate.format, down_slice(I, w->gate.format), 1) > kStageMax)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "ffn_dense: hidden size %d too large for the staged GEMV", H);
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: hidden size %d too large for the staged GEMV", who, H);
   Carve c{nullptr};
   carve_dense(c, M, H, I);
   if ((rc = check_ws(ws, ws_bytes, c.off)) != MOEFFN_OK) return rc;
@@ -515,7 +589,8 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int splits = 0;
   bool tail_done = false;
-  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits, residual, &tail_done)) != MOEFFN_OK) return rc;
+  if ((rc = run_dense_ffn(*w, x, M, H, I, act, d, s, &splits, residual, &tail_done, norm_w, eps)) != MOEFFN_OK)
+    return rc;
   if (tail_done) return MOEFFN_OK;
   TailArgs t{};
   t.mode = TAIL_RESIDUAL;
@@ -530,6 +605,20 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
     MOEFFN_CHECK_CUDA(launch_tail(t, s), "residual tail launch");
   }
   return MOEFFN_OK;
+}
+
+}  // namespace
+
+int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M, int act, void* ws,
+              size_t ws_bytes, moeffn_stream_t stream) {
+  if (x == nullptr) return fail(MOEFFN_ERR_INVALID, "ffn_dense: null pointer");
+  return dense_entry("ffn_dense", w, x, nullptr, 0.f, residual, M, act, ws, ws_bytes, stream);
+}
+
+int ffn_dense_prenorm(const moeffn_ffn* w, const uint16_t* norm_w, float eps, uint16_t* residual, int M, int act,
+                      void* ws, size_t ws_bytes, moeffn_stream_t stream) {
+  if (norm_w == nullptr) return fail(MOEFFN_ERR_INVALID, "ffn_dense_prenorm: null norm weight");
+  return dense_entry("ffn_dense_prenorm", w, nullptr, norm_w, eps, residual, M, act, ws, ws_bytes, stream);
 }
 
 int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* norm_w, float eps, uint16_t* h1_out,
@@ -665,12 +754,20 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
     if ((rc = check_ffn(*desc->shared, "shared", H, Is)) != MOEFFN_OK) return rc;
     if (desc->shared->gate.format != MOEFFN_Q_INT4_AFFINE_G32)
       return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: the shared expert must be INT4-affine like the routed ones");
-    if (desc->shared_gate == nullptr || desc->shared_gate->q == nullptr || desc->shared_gate->format != MOEFFN_BF16 ||
-        desc->shared_gate->cols != H || desc->shared_gate->rows != 1 || !aligned16(desc->shared_gate->q))
+    if (desc->shared_post_norm != nullptr) {   // Gemma form: normed, ungated shared branch
+      if (desc->shared_gate != nullptr)
+        return fail(MOEFFN_ERR_INVALID, "moe_plan_create: the Gemma form (shared_post_norm) has no shared_gate");
+      if (!aligned16(desc->shared_post_norm) || !(desc->shared_post_norm_eps >= 0.0f))
+        return fail(MOEFFN_ERR_INVALID, "moe_plan_create: shared_post_norm not 16-byte aligned or eps < 0");
+    } else if (desc->shared_gate == nullptr || desc->shared_gate->q == nullptr || desc->shared_gate->format != MOEFFN_BF16 ||
+               desc->shared_gate->cols != H || desc->shared_gate->rows != 1 || !aligned16(desc->shared_gate->q)) {
       return fail(MOEFFN_ERR_INVALID, "moe_plan_create: shared expert needs a BF16 [1][H] 16-byte aligned shared_gate");
-  } else if (desc->shared_gate != nullptr) {
-    return fail(MOEFFN_ERR_INVALID, "moe_plan_create: shared_gate without a shared expert");
+    }
+  } else if (desc->shared_gate != nullptr || desc->shared_post_norm != nullptr) {
+    return fail(MOEFFN_ERR_INVALID, "moe_plan_create: shared_gate / shared_post_norm without a shared expert");
   }
+  if (desc->expert_scale != nullptr && (reinterpret_cast<uintptr_t>(desc->expert_scale) & 3u) != 0)
+    return fail(MOEFFN_ERR_INVALID, "moe_plan_create: expert_scale not 4-byte aligned");
   if (gemv_stage_bytes(MOEFFN_Q_INT4_AFFINE_G32, H, 1) > kStageMax)
     return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: hidden size %d too large", H);
   auto* p = new moeffn_moe_plan();
@@ -683,8 +780,11 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   if (p->has_shared) p->tma = p->tma && tma_ok(*desc->shared);
   if (p->has_shared) {
     p->shared = *desc->shared;
-    p->w_sg = static_cast<const uint16_t*>(desc->shared_gate->q);
+    p->w_sg = desc->shared_gate != nullptr ? static_cast<const uint16_t*>(desc->shared_gate->q) : nullptr;
   }
+  p->expert_scale = desc->expert_scale;
+  p->shared_post_norm = desc->shared_post_norm;
+  p->shared_post_norm_eps = desc->shared_post_norm_eps;
   cudaError_t e1 = cudaMalloc(&p->d_gate, sizeof(QW) * E);
   cudaError_t e2 = cudaMalloc(&p->d_up, sizeof(QW) * E);
   cudaError_t e3 = cudaMalloc(&p->d_down, sizeof(QW) * E);
@@ -727,20 +827,16 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   if (tc && p->has_shared) tc = tc_ok(*desc->shared);
   if (tc) {
     std::vector<TcMaps> tg(E), tu(E), td(E);
-    p->tc_fe = tc_gateup_feat(Ie);
-    p->tc_fs = p->has_shared ? tc_gateup_feat(Is) : 8;
-    p->tc_rd = tc_down_rows(H);
-    const int fe = p->tc_fe, fs = p->tc_fs, rd = p->tc_rd;
     bool ok = true;
     for (int e = 0; e < E && ok; ++e) {
-      ok = encode_tc_weight_maps(&tg[e], MOEFFN_Q_INT4_AFFINE_G32, g[e], Ie, H, fe) == cudaSuccess &&
-           encode_tc_weight_maps(&tu[e], MOEFFN_Q_INT4_AFFINE_G32, u[e], Ie, H, fe) == cudaSuccess &&
-           encode_tc_weight_maps(&td[e], MOEFFN_Q_INT4_AFFINE_G32, d[e], H, Ie, rd) == cudaSuccess;
+      ok = encode_tc_weight_maps(&tg[e], MOEFFN_Q_INT4_AFFINE_G32, g[e], Ie, H) == cudaSuccess &&
+           encode_tc_weight_maps(&tu[e], MOEFFN_Q_INT4_AFFINE_G32, u[e], Ie, H) == cudaSuccess &&
+           encode_tc_weight_maps(&td[e], MOEFFN_Q_INT4_AFFINE_G32, d[e], H, Ie) == cudaSuccess;
     }
     if (ok && p->has_shared) {
-      ok = encode_tc_weight_maps(&p->tc_sg, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.gate), Is, H, fs) == cudaSuccess &&
-           encode_tc_weight_maps(&p->tc_su, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.up), Is, H, fs) == cudaSuccess &&
-           encode_tc_weight_maps(&p->tc_sd, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.down), H, Is, rd) == cudaSuccess;
+      ok = encode_tc_weight_maps(&p->tc_sg, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.gate), Is, H) == cudaSuccess &&
+           encode_tc_weight_maps(&p->tc_su, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.up), Is, H) == cudaSuccess &&
+           encode_tc_weight_maps(&p->tc_sd, MOEFFN_Q_INT4_AFFINE_G32, to_qw(p->shared.down), H, Is) == cudaSuccess;
     }
     const size_t bytes = sizeof(TcMaps) * E;
     if (!ok || cudaMalloc(&p->d_tc_gate, bytes) != cudaSuccess || cudaMalloc(&p->d_tc_up, bytes) != cudaSuccess ||
@@ -778,13 +874,23 @@ size_t moe_workspace_bytes(const moeffn_moe_plan* p, int M) {
   return c.off;
 }
 
-int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, int32_t* topk_idx_out, void* ws,
-              size_t ws_bytes, moeffn_stream_t stream) {
+namespace {
+
+// moe_layer and moe_layer_prenorm: with norm_w, x is null and the input is
+// m = rms_norm(residual, norm_w), formed by the router kernel.
+int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint16_t* norm_w, float eps,
+              uint16_t* residual, int M, int32_t* topk_idx_out, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
   g_last_error.clear();
-  if (p == nullptr || x == nullptr || residual == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_layer: null pointer");
-  if (M < 1) return fail(MOEFFN_ERR_INVALID, "moe_layer: M=%d", M);
-  if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "moe_layer: x/residual not 16-byte aligned");
-  if (x == residual) return fail(MOEFFN_ERR_INVALID, "moe_layer: x aliases residual");
+  if (p == nullptr || residual == nullptr || (x == nullptr && norm_w == nullptr))
+    return fail(MOEFFN_ERR_INVALID, "%s: null pointer", who);
+  if (M < 1) return fail(MOEFFN_ERR_INVALID, "%s: M=%d", who, M);
+  if (norm_w != nullptr) {
+    if (!aligned16(norm_w)) return fail(MOEFFN_ERR_INVALID, "%s: norm weight not 16-byte aligned", who);
+    if (!(eps >= 0.0f)) return fail(MOEFFN_ERR_INVALID, "%s: eps must be >= 0", who);
+  }
+  if ((x != nullptr && !aligned16(x)) || !aligned16(residual))
+    return fail(MOEFFN_ERR_INVALID, "%s: x/residual not 16-byte aligned", who);
+  if (x == residual) return fail(MOEFFN_ERR_INVALID, "%s: x aliases residual", who);
   const int E = p->E, k = p->k, H = p->H, Ie = p->Ie, Is = p->Is;
   Carve c{nullptr};
   carve_moe(c, M, H, Ie, Is, E, k);
@@ -798,13 +904,19 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   RouterArgs ra{};
   ra.router = p->router;
   ra.router_f32 = p->router_fmt == MOEFFN_F32;
-  ra.w_sg = p->has_shared ? p->w_sg : nullptr;
-  ra.x = x;
+  ra.w_sg = p->has_shared ? p->w_sg : nullptr;   // null in the Gemma form (no gate)
+  ra.x = norm_w != nullptr ? residual : x;
   ra.M = M;
   ra.H = H;
   ra.E = E;
   ra.logits = w.logits;
   ra.gate_logit = w.gate_logit;
+  if (norm_w != nullptr) {   // the router kernel forms m for every later step
+    ra.norm_w = norm_w;
+    ra.eps = eps;
+    ra.m_out = w.m;
+    x = w.m;
+  }
   {
     ProfScope ps("router_logits", s);
     MOEFFN_CHECK_CUDA(launch_router_logits(ra, s), "router launch");
@@ -822,6 +934,7 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   rt.offsets = w.offsets;
   rt.union_list = w.union_list;
   rt.n_union = w.n_union;
+  rt.scale = p->expert_scale;
   {
     ProfScope ps("route_topk", s);
     MOEFFN_CHECK_CUDA(launch_route(rt, s), "route launch");
@@ -844,20 +957,18 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
       ProfScope ps("gather_rows", s);
       MOEFFN_CHECK_CUDA(launch_gather_rows(ga, s), "gather launch");
     }
-    // One CTA should cover a whole expert's token rows, since a second CTA
-    // would dequantize every weight of the expert again: two 128-row token
-    // tiles per CTA once the expected load, plus half again for the routing
-    // spread, passes 128.
+    // One CTA should cover a whole expert's token rows, since a second token
+    // tile dequantizes every weight of the expert again: the token tile is
+    // sized for the mean load per expert plus half again for the routing
+    // spread (an expert holds at most M rows).
     const int per_expert = std::max(1, P / std::min(E, P));
-    const int mt = tc_mt_for(per_expert + per_expert / 2), tpc = tc_tokens_per_cta(mt);
-    const int tt = (M + tpc - 1) / tpc;   // an expert has at most M token rows
+    const int ntile = tc_ntile_for(std::min(M, per_expert + per_expert / 2 + 1));
+    const int tt = (M + ntile - 1) / ntile;
     TcGemmArgs g{};
     g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
     g.act = p->act;
     g.mode = TC_GATEUP;
-    g.mt = mt;
-    g.tile = p->tc_fe;
-    g.tile_s = p->tc_fs;
+    g.ntile = ntile;
     g.N = Ie;
     g.K = H;
     g.Ns = Is;
@@ -876,9 +987,9 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     g.out_act_s = w.acts_s;
     g.ks_len = H;
     g.token_tiles = tt;
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, w.xg, P, H), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap_s, x, M, H), "tensor map encode");
-    const int rt1 = std::max((Ie + p->tc_fe - 1) / p->tc_fe, Is > 0 ? (Is + p->tc_fs - 1) / p->tc_fs : 0);
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap, w.xg, P, H, ntile), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&g.xmap_s, x, M, H, ntile), "tensor map encode");
+    const int rt1 = (std::max(Ie, Is) + kTcGateUpFeat - 1) / kTcGateUpFeat;
     {
       ProfScope ps("phase1_gateup_gemm_tc", s);
       MOEFFN_CHECK_CUDA(launch_tc_gemm(g, rt1, 1, jobs, s), "phase-1 GEMM launch");
@@ -886,9 +997,7 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     TcGemmArgs d{};
     d.fmt = MOEFFN_Q_INT4_AFFINE_G32;
     d.mode = TC_DOWN;
-    d.mt = mt;
-    d.tile = p->tc_rd;
-    d.tile_s = p->tc_rd;
+    d.ntile = ntile;
     d.N = H;
     d.K = Ie;
     d.Ns = H;
@@ -904,9 +1013,9 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     d.out_d = w.d;
     d.out_d_s = w.d_s;
     d.token_tiles = tt;
-    const int row_tiles = (H + p->tc_rd - 1) / p->tc_rd;
-    const int active = std::max(1, std::min(E, P)) * std::max(1, (per_expert + tpc - 1) / tpc);
-    const int want = (2 * kSMs + row_tiles * active - 1) / (row_tiles * active);
+    const int row_tiles = (H + kTcDownRows - 1) / kTcDownRows;
+    const int active = std::max(1, std::min(E, P)) * std::max(1, (per_expert + ntile - 1) / ntile);
+    const int want = (kSMs + row_tiles * active - 1) / (row_tiles * active);
     d.ks_len = tc_down_slice(Ie, MOEFFN_Q_INT4_AFFINE_G32, want, sp.routed);
     tc_splits_r = (Ie + d.ks_len - 1) / d.ks_len;
     tc_splits_s = Is > 0 ? (Is + d.ks_len - 1) / d.ks_len : 0;
@@ -915,8 +1024,8 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
       tc_splits_r = splits_r;
       tc_splits_s = splits_sh;
     }
-    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, P, Ie), "tensor map encode");
-    if (Is > 0) MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap_s, w.acts_s, M, Is), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, P, Ie, ntile), "tensor map encode");
+    if (Is > 0) MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap_s, w.acts_s, M, Is, ntile), "tensor map encode");
     {
       ProfScope ps("phase2_down_gemm_tc", s);
       MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, std::max(tc_splits_r, tc_splits_s), jobs, s),
@@ -1052,7 +1161,9 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
   }
 
   TailArgs t{};
-  t.mode = TAIL_MOE;
+  t.mode = p->shared_post_norm != nullptr ? TAIL_MOE_GEMMA : TAIL_MOE;
+  t.norm_w = p->shared_post_norm;
+  t.eps = p->shared_post_norm_eps;
   t.M = M;
   t.N = H;
   t.d = w.d;
@@ -1070,6 +1181,20 @@ int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, 
     MOEFFN_CHECK_CUDA(launch_tail(t, s), "moe tail launch");
   }
   return MOEFFN_OK;
+}
+
+}  // namespace
+
+int moe_layer(moeffn_moe_plan* p, const uint16_t* x, uint16_t* residual, int M, int32_t* topk_idx_out, void* ws,
+              size_t ws_bytes, moeffn_stream_t stream) {
+  if (x == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_layer: null pointer");
+  return moe_entry("moe_layer", p, x, nullptr, 0.f, residual, M, topk_idx_out, ws, ws_bytes, stream);
+}
+
+int moe_layer_prenorm(moeffn_moe_plan* p, const uint16_t* norm_w, float eps, uint16_t* residual, int M,
+                      int32_t* topk_idx_out, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
+  if (norm_w == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_layer_prenorm: null norm weight");
+  return moe_entry("moe_layer_prenorm", p, nullptr, norm_w, eps, residual, M, topk_idx_out, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -8,17 +8,20 @@ namespace moeffn {
 
 enum : int { TC_GATEUP = 2, TC_DOWN = 1 };
 
-// Tensor maps of one quantized matrix for the GEMM: codes (uint8, 128-byte
-// swizzled boxes of [tile rows][128 bytes]), INT4 scales and mins (u16 boxes
-// of [tile rows][8 groups]). The box height is the tile's weight rows per
-// matrix: F for gate and up (GATEUP), R for down.
+// Weight rows of one MMA A tile, and token rows (MMA N) one CTA covers at most.
+constexpr int kTcRowsA = 128;
+constexpr int kTcMaxTok = 192;
+
+// Tensor maps of one quantized matrix for the GEMM, boxes of kTcRowsA rows:
+// codes (uint8, 128-byte swizzled [128 rows][128 bytes]), INT4 scales and
+// mins (u16 [128 rows][8 groups]).
 struct TcMaps {
   CUtensorMap codes, scale, mn;
 };
 
 struct TcGemmArgs {
-  CUtensorMap xmap;            // A operand rows (dense / routed jobs): bf16 [rows][K], boxes [128][64]
-  CUtensorMap xmap_s;          // A operand rows of the shared job
+  CUtensorMap xmap;            // B operand rows (dense / routed jobs): bf16 [rows][K], boxes [ntile][64]
+  CUtensorMap xmap_s;          // B operand rows of the shared job
   TcMaps w0, w1;               // dense mode: gate, up (GATEUP) or down (w0)
   const TcMaps* tab0;          // grouped mode: per expert [E]
   const TcMaps* tab1;
@@ -26,8 +29,7 @@ struct TcGemmArgs {
   const __half* rscale0;       // INT8 dense: per-row scales of w0 / w1
   const __half* rscale1;
   int fmt, act, mode;
-  int mt;                      // 128-row token tiles per CTA (1 or 2)
-  int tile, tile_s;            // features per tile (GATEUP, <= 128) or output rows (DOWN, <= 256)
+  int ntile;                   // token rows per CTA tile (multiple of 16, <= kTcMaxTok; the maps' box height)
   int N, K, Ns, Ks;            // dense / routed and shared shapes (rows, reduction)
   int M;
   const int* offsets;          // null: dense mode
@@ -45,17 +47,16 @@ struct TcGemmArgs {
 
 // K covered by one weight stage: 256 codes (INT4) or 128 (INT8).
 inline int tc_k_tile(int fmt) { return fmt == FMT_INT4_G32 ? 256 : 128; }
-// Features per GATEUP tile for an intermediate size I, rows per DOWN tile for
-// an output size H.
-int tc_gateup_feat(int I);
-int tc_down_rows(int H);
-// Token tiles per CTA for an expected token count per weight matrix, and the
-// token rows one CTA covers.
-int tc_mt_for(int tokens);
-int tc_tokens_per_cta(int mt);
+// Output features per CTA (GATEUP: 128 gate rows and the same 128 up rows) and
+// output rows per CTA (DOWN: two tiles of 128).
+constexpr int kTcGateUpFeat = kTcRowsA;
+constexpr int kTcDownRows = 2 * kTcRowsA;
+// Token rows per CTA tile for `tokens` rows in a job: the fewest tiles of at
+// most kTcMaxTok, balanced, rounded up to the MMA's N granule of 16.
+int tc_ntile_for(int tokens);
 
-cudaError_t encode_tc_weight_maps(TcMaps* m, int fmt, const QW& w, int N, int K, int box_rows);
-cudaError_t encode_tc_x_map(CUtensorMap* m, const uint16_t* x, int rows, int K);
+cudaError_t encode_tc_weight_maps(TcMaps* m, int fmt, const QW& w, int N, int K);
+cudaError_t encode_tc_x_map(CUtensorMap* m, const uint16_t* x, int rows, int K, int ntile);
 cudaError_t launch_tc_gemm(const TcGemmArgs& a, int row_tiles, int splits, int jobs, cudaStream_t s);
 unsigned int tc_gemm_fault_flags(bool clear);
 

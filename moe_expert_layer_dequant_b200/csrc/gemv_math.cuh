@@ -2,6 +2,7 @@
 // codes times staged activations summed exactly in int32 with DP2A.
 #pragma once
 #include "common.cuh"
+#include "norm.cuh"
 
 namespace moeffn {
 
@@ -73,9 +74,12 @@ struct Codes<FMT_INT8_ROW> {
 // Stages one chunk of a bf16 activation row (p: the chunk's first element,
 // 16-byte aligned; null for a zero pad row): the int16 values in code order
 // at dst, the chunk's power-of-two factor in *xf and (INT4) its plain sum in
-// *xsum, the sum the min term of the affine format multiplies.
+// *xsum, the sum the min term of the affine format multiplies. With `wn`
+// (the same chunk of an RMSNorm weight) the chunk is first normalized:
+// x -> bf16(x * inv_rms * w).
 template <int FMT>
-__device__ __forceinline__ void stage_chunk(const uint16_t* p, uint8_t* dst, float* xf, float* xsum) {
+__device__ __forceinline__ void stage_chunk(const uint16_t* p, uint8_t* dst, float* xf, float* xsum,
+                                            const uint16_t* wn = nullptr, float inv_rms = 0.f) {
   using C = Codes<FMT>;
   uint16_t v[C::kChunk];
   if (p != nullptr) {
@@ -87,6 +91,18 @@ __device__ __forceinline__ void stage_chunk(const uint16_t* p, uint8_t* dst, flo
       for (int j = 0; j < 4; ++j) {
         v[8 * q + 2 * j] = (uint16_t)(w[j] & 0xFFFFu);
         v[8 * q + 2 * j + 1] = (uint16_t)(w[j] >> 16);
+      }
+    }
+    if (wn != nullptr) {
+#pragma unroll
+      for (int q = 0; q < C::kChunk / 8; ++q) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(wn) + q);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[8 * q + 2 * j] = prenorm_elem(v[8 * q + 2 * j], (uint16_t)(w[j] & 0xFFFFu), inv_rms);
+          v[8 * q + 2 * j + 1] = prenorm_elem(v[8 * q + 2 * j + 1], (uint16_t)(w[j] >> 16), inv_rms);
+        }
       }
     }
   } else {

@@ -60,6 +60,11 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
+// Barrier of one consumer group (ids 2.. for the groups).
+__device__ __forceinline__ void group_sync(int grp, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(2 + grp), "r"(nthreads) : "memory");
+}
+
 // NC consumer warps per group, G groups: group g takes the stages s with
 // s % G == g, one row of the stage per warp (R = NC rows per stage). The ring
 // depth S is a multiple of G, so every slot is waited on by one group only,
@@ -78,7 +83,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   // lists the routing kernels write) wait for it first.
   const bool early = a.offsets == nullptr;
   if (!early) pdl_wait();
-  if (a.stages % G != 0 || a.stages > 8) {   // ring depth the host must not choose
+  if (a.stages < G || a.stages % G != 0 || a.stages > 8) {   // ring depth the host must not choose
     if (threadIdx.x == 0) atomicOr(&g_fault_flags, 2u);
     return;
   }
@@ -113,7 +118,8 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   float* xf = reinterpret_cast<float*>(xi + (size_t)tok_rows * tok_stride);  // [tok_rows][nch] factors
   float* xsum = xf + (size_t)tok_rows * nch;                        // [tok_rows][nch] (INT4)
   const size_t x_bytes = ((size_t)tok_rows * (tok_stride + 4 * nch + (kInt4 ? 4 * nch : 0)) + 127) / 128 * 128;
-  uint8_t* stage0 = smem + 128 + x_bytes;
+  // then the group's row-sum exchange buffers [G][2][NC][R * NM * MT] floats
+  uint8_t* stage0 = smem + 128 + x_bytes + gemv_red_bytes(NM, MT, G);
   const size_t stage_bytes = (size_t)NM * R * (cs + 4 * gst);
   // within a stage: codes [NM][R][cs], scales [NM][R][gst], mins [NM][R][gst]
 
@@ -136,12 +142,14 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   // The next kernel in the stream may be scheduled now; it waits for this
   // grid's completion before reading what this grid writes.
   pdl_launch_dependents();
+  const unsigned long long wait_ns = a.wait_ns != 0 ? a.wait_ns : kWaitLimitNs;
   if (warp == NC * G) {
     // ---------------- producer ----------------
     if (lane == 0) {
       for (int s = 0; s < total; ++s) {
         const int slot = s % S, use = s / S;
-        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1)) break;
+        if (a.inject_stop > 0 && s >= a.inject_stop - 1) break;   // injected producer failure (tests)
+        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, wait_ns)) break;
         const int n0 = r0 + (s % row_stages) * R;
         const int nr = min(R, r1 - n0);
         uint8_t* st = stage0 + (size_t)slot * stage_bytes;
@@ -179,17 +187,56 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   }
 
   // ---------------- consumers ----------------
+  // Lane mapping: lane l of a warp owns chunk 32 b + l of the K slice (b a
+  // K block of 32 chunks); the warps of a group split the K blocks and, when
+  // there are fewer K blocks than warps, the stage's rows (row phases: warp
+  // phase j takes rows j, j + P, ...). A lane loads its chunk's staged
+  // activations once per stage and token pass and multiplies them with the
+  // codes of every row it owns; the row sums are then reduced across the
+  // warp (transposed butterfly), across the group's warps through shared
+  // memory (fixed order) and written by one warp per row.
   if (early) pdl_wait();
   const int nthreads = NC * G * 32;
   if (a.zero_cnt != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
     for (int i = threadIdx.x; i < a.zero_n; i += nthreads) a.zero_cnt[i] = 0;
-  const int grp = warp / NC, wr = warp - grp * NC;  // group, row of the stage
+  const int grp = warp / NC, wr = warp - grp * NC;  // group, warp within the group
   const uint16_t* src = job.shared ? a.x_s : a.x;
   const int ld = job.shared ? job.K : a.ld_x;
+  const int nkb = (nch + 31) / 32;                  // K blocks of 32 chunks
+  const int P = nkb >= NC ? 1 : NC / nkb;           // row phases
+  const int wj = P > 1 ? wr / nkb : 0;              // this warp's row phase
+  const int wb = P > 1 ? wr % nkb : wr;             // its first K block
+  const int bstep = P > 1 ? nkb : NC;               // K blocks between its blocks
+  const bool wactive = wj < P;
+  constexpr int V = R * NM * MT;                    // row sums per stage and token pass
+  float* red = reinterpret_cast<float*>(smem + 128 + x_bytes) + (size_t)grp * 2 * NC * V;   // [G][2][NC][V]
+  const int mn_off = NM * R * gst * 2;              // mins follow the scales in a stage
   bool dead = false;
+  int pass = 0;                                     // stage passes of this group (red buffer parity)
   for (int tb = 0, tbi = 0; tb < job.ntok; tb += a.stage_tokens, ++tbi) {
     const int tn = min(a.stage_tokens, job.ntok - tb);
     consumer_sync(nthreads);
+    // Input norm folded in (dense gate/up: the job's whole row is this CTA's
+    // K range): inv_rms of every staged token row, from per-warp sums of
+    // squares added in warp order. The exchange buffers are free here.
+    const bool norm = a.norm_w != nullptr;
+    float* inv_rms = reinterpret_cast<float*>(smem + 128 + x_bytes);   // [tok_rows], then [tok_rows][warps] partial sums
+    if (norm) {
+      const int nw = nthreads / 32;
+      float* ssp = inv_rms + tok_rows;
+      for (int r = 0; r < tn; ++r) {
+        float ss = row_sumsq_part(src + (size_t)(job.slot0 + tb + r) * ld, job.K, threadIdx.x, nthreads);
+        ss = warp_sum(ss);
+        if (lane == 0) ssp[r * nw + warp] = ss;
+      }
+      consumer_sync(nthreads);
+      if (threadIdx.x < tn) {
+        float ss = 0.f;
+        for (int w = 0; w < nw; ++w) ss += ssp[threadIdx.x * nw + w];
+        inv_rms[threadIdx.x] = inv_rms_of(ss, job.K, a.eps);
+      }
+      consumer_sync(nthreads);
+    }
     // Stage token rows tb..tb+tn (K slice) chunk by chunk: int16 fixed point,
     // the chunk's power-of-two factor and (INT4) its plain sum; zero pad rows.
     for (int i = threadIdx.x; i < tok_rows * nch; i += nthreads) {
@@ -199,116 +246,117 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
         const int row = job.gather ? a.perm[job.slot0 + tb + r] / a.topk : job.slot0 + tb + r;
         p = src + (size_t)row * ld + k0 + c * C::kChunk;
       }
-      stage_chunk<FMT>(p, xi + r * tok_stride + c * C::kStageBytes, &xf[r * nch + c], &xsum[r * nch + c]);
+      stage_chunk<FMT>(p, xi + r * tok_stride + c * C::kStageBytes, &xf[r * nch + c], &xsum[r * nch + c],
+                       (norm && p != nullptr) ? a.norm_w + k0 + c * C::kChunk : nullptr,
+                       (norm && p != nullptr) ? inv_rms[r] : 0.f);
     }
     consumer_sync(nthreads);
 
     for (int rs = grp; rs < row_stages; rs += G) {
       const int s = tbi * row_stages + rs;
       const int slot = s % S, use = s / S;
-      const int n = r0 + rs * R + wr;
-      float row_scale[NM];
-      if (!kInt4 && n < r1) {
-#pragma unroll
-        for (int i = 0; i < NM; ++i) row_scale[i] = __half2float(__ldg(job.m[i].scale + n));
-      }
+      const int n0 = r0 + rs * R;                   // first row of the stage
       // After a timed-out wait (a fault already recorded) the warp stops
       // computing but still takes part in every barrier below.
-      if (!dead && !mbar_wait(&full[slot], use & 1)) dead = true;
-      if (!dead && n < r1) {
-        // 32-bit byte offsets from the stage start (shared memory).
-        const uint8_t* st = stage0 + slot * (int)stage_bytes;
-        int o_code[NM], o_sc[NM];
+      if (!dead && !mbar_wait(&full[slot], use & 1, wait_ns)) dead = true;
+      dead = __any_sync(0xffffffffu, dead);
+      const uint8_t* st = stage0 + slot * (int)stage_bytes;
+      for (int tc = 0; tc < tn; tc += MT, ++pass) {
+        float part[V];
 #pragma unroll
-        for (int i = 0; i < NM; ++i) {
-          o_code[i] = (i * R + wr) * cs + lane * 16;
-          o_sc[i] = NM * R * cs + ((i * R + wr) * gst + lane) * 2;
-        }
-        const int mn_off = NM * R * gst * 2;   // mins follow the scales
-        for (int tc = 0; tc < tn; tc += MT) {
-          float acc[NM][MT];
-#pragma unroll
-          for (int i = 0; i < NM; ++i)
-#pragma unroll
-            for (int t = 0; t < MT; ++t) acc[i][t] = 0.f;
-          int ox = tc * tok_stride + lane * C::kStageBytes;   // staged activations
-          int of = tc * nch + lane;                            // factors / sums
-          int oc = 0, og = 0;                                  // code / scale advance
-          for (int c = lane; c < nch; c += 32, ox += 32 * C::kStageBytes, of += 32, oc += 512, og += 64) {
-            uint4 wv[NM];
-            float sc[NM], mn[NM];
-#pragma unroll
-            for (int i = 0; i < NM; ++i) {
-              wv[i] = *reinterpret_cast<const uint4*>(st + o_code[i] + oc);
-              if (kInt4) {
-                sc[i] = __half2float(*reinterpret_cast<const __half*>(st + o_sc[i] + og));
-                mn[i] = __half2float(*reinterpret_cast<const __half*>(st + o_sc[i] + og + mn_off));
-              }
-            }
-            int p0[NM][MT], p1[NM][MT];
-#pragma unroll
-            for (int i = 0; i < NM; ++i)
-#pragma unroll
-              for (int t = 0; t < MT; ++t) p0[i][t] = p1[i][t] = 0;
-            if (kInt4) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-#pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                  const uint4 x4 = *reinterpret_cast<const uint4*>(xi + ox + t * tok_stride + q * 16);
-#pragma unroll
-                  for (int i = 0; i < NM; ++i) {
-                    const uint32_t w = q == 0 ? wv[i].x : q == 1 ? wv[i].y : q == 2 ? wv[i].z : wv[i].w;
-                    Codes<FMT_INT4_G32>::dot_word(w, x4, p0[i][t], p1[i][t]);
-                  }
-                }
-              }
-            } else {
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                for (int t = 0; t < MT; ++t) {
-                  const uint4 x4 = *reinterpret_cast<const uint4*>(xi + ox + t * tok_stride + h * 16);
-#pragma unroll
-                  for (int i = 0; i < NM; ++i) {
-                    const uint32_t w0 = h == 0 ? wv[i].x : wv[i].z, w1 = h == 0 ? wv[i].y : wv[i].w;
-                    Codes<FMT_INT8_ROW>::dot_word(w0, w1, x4, p0[i][t], p1[i][t]);
-                  }
-                }
-              }
-            }
+        for (int v = 0; v < V; ++v) part[v] = 0.f;
+        if (!dead && wactive) {
+          for (int b = wb; b < nkb; b += bstep) {
+            const int c = 32 * b + lane;
+            if (c >= nch) continue;
+            uint4 x4[MT][C::kChunk / 8];
+            float f[MT], X[MT];
 #pragma unroll
             for (int t = 0; t < MT; ++t) {
-              const float f = xf[of + t * nch];
-              const float X = kInt4 ? xsum[of + t * nch] : 0.f;
+#pragma unroll
+              for (int q = 0; q < C::kChunk / 8; ++q)
+                x4[t][q] = *reinterpret_cast<const uint4*>(xi + (tc + t) * tok_stride + c * C::kStageBytes + q * 16);
+              f[t] = xf[(tc + t) * nch + c];
+              X[t] = kInt4 ? xsum[(tc + t) * nch + c] : 0.f;
+            }
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+              if (r % P != wj) continue;            // rows of this warp's phase
 #pragma unroll
               for (int i = 0; i < NM; ++i) {
-                const float P = (float)(p0[i][t] + p1[i][t]);   // exact below 2^24
-                // sum_k (q_k s + m) x_k = s * 2^(e-14) * sum_k q_k xi_k + m * sum_k x_k
-                acc[i][t] = kInt4 ? fmaf(sc[i] * f, P, fmaf(mn[i], X, acc[i][t])) : fmaf(f, P, acc[i][t]);
+                const uint4 wv = *reinterpret_cast<const uint4*>(st + (size_t)(i * R + r) * cs + c * 16);
+                float sc = 0.f, mn = 0.f;
+                if (kInt4) {
+                  const int o = NM * R * cs + ((i * R + r) * gst + c) * 2;
+                  sc = __half2float(*reinterpret_cast<const __half*>(st + o));
+                  mn = __half2float(*reinterpret_cast<const __half*>(st + o + mn_off));
+                }
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                  int p0 = 0, p1 = 0;
+                  if (kInt4) {
+                    Codes<FMT_INT4_G32>::dot_word(wv.x, x4[t][0], p0, p1);
+                    Codes<FMT_INT4_G32>::dot_word(wv.y, x4[t][1 % (C::kChunk / 8)], p0, p1);
+                    Codes<FMT_INT4_G32>::dot_word(wv.z, x4[t][2 % (C::kChunk / 8)], p0, p1);
+                    Codes<FMT_INT4_G32>::dot_word(wv.w, x4[t][3 % (C::kChunk / 8)], p0, p1);
+                  } else {
+                    Codes<FMT_INT8_ROW>::dot_word(wv.x, wv.y, x4[t][0], p0, p1);
+                    Codes<FMT_INT8_ROW>::dot_word(wv.z, wv.w, x4[t][1 % (C::kChunk / 8)], p0, p1);
+                  }
+                  const float Pq = (float)(p0 + p1);   // exact below 2^24
+                  // sum_k (q_k s + m) x_k = s * 2^(e-14) * sum_k q_k xi_k + m * sum_k x_k
+                  float& acc = part[(r * NM + i) * MT + t];
+                  acc = kInt4 ? fmaf(sc * f[t], Pq, fmaf(mn, X[t], acc)) : fmaf(f[t], Pq, acc);
+                }
               }
             }
           }
-          // epilogue
+        }
+        // Warp sums: a transposed butterfly leaves lane l with value
+        // l >> (5 - log2 V) summed over the warp's 32 lanes.
+        int live = V;
 #pragma unroll
-          for (int t = 0; t < MT; ++t) {
-            float v[NM];
+        for (int o = 16; o >= 1; o >>= 1) {
+          if (live > 1) {
+            const bool upper = (lane & o) != 0;
 #pragma unroll
-            for (int i = 0; i < NM; ++i) {
-              v[i] = warp_sum(acc[i][t]);
-              if (!kInt4) v[i] *= row_scale[i];
-            }
-            const int tok = tb + tc + t;
-            if (lane == 0 && tok < tn + tb) {
-              const int slot_out = job.slot0 + tok;
-              if (NM == 2) {
-                uint16_t* out = job.shared ? a.out_act_s : a.out_act;
-                out[(size_t)slot_out * job.N + n] = float_to_bf16_bits(gated_act(v[0], v[NM - 1], a.act));
-              } else {
-                float* d = job.shared ? a.out_d_s : a.out_d;
-                const int nslots = job.shared ? a.M : a.slots;
-                d[((size_t)blockIdx.y * nslots + slot_out) * job.N + n] = v[0];
+            for (int k = 0; k < V / 2; ++k) {
+              if (k < live / 2) {
+                const float send = upper ? part[k] : part[k + live / 2];
+                const float keep = upper ? part[k + live / 2] : part[k];
+                part[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
               }
+            }
+            live >>= 1;
+          } else {
+            part[0] += __shfl_xor_sync(0xffffffffu, part[0], o);
+          }
+        }
+        constexpr int kLog2V = V == 8 ? 3 : (V == 16 ? 4 : 5);
+        float* rb = red + (size_t)(pass & 1) * NC * V;
+        if ((lane & ((1 << (5 - kLog2V)) - 1)) == 0) rb[wr * V + (lane >> (5 - kLog2V))] = part[0];
+        group_sync(grp, NC * 32);
+        // Row r of the stage: warp r adds the group's warp sums in warp order.
+        const int n = n0 + wr;
+        if (!dead && n < r1 && lane < NM * MT) {
+          const int i = lane / MT, t = lane % MT;
+          float v = 0.f;
+          for (int w = 0; w < NC; ++w) v += rb[w * V + (wr * NM + i) * MT + t];
+          if (!kInt4) v *= __half2float(__ldg(job.m[i].scale + n));
+          float other = 0.f;   // NM == 2: the up sum of the same token, from lane MT + t
+          if (NM == 2) other = __shfl_down_sync((1u << (NM * MT)) - 1u, v, MT);
+          const int tok = tb + tc + t;
+          if (tok < tn + tb) {
+            const int slot_out = job.slot0 + tok;
+            if (NM == 2) {
+              if (i == 0) {
+                uint16_t* out = job.shared ? a.out_act_s : a.out_act;
+                out[(size_t)slot_out * job.N + n] = float_to_bf16_bits(gated_act(v, other, a.act));
+              }
+            } else {
+              float* d = job.shared ? a.out_d_s : a.out_d;
+              const int nslots = job.shared ? a.M : a.slots;
+              d[((size_t)blockIdx.y * nslots + slot_out) * job.N + n] = v;
             }
           }
         }
@@ -368,11 +416,12 @@ size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
 
 size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages) {
   const bool i4 = fmt == FMT_INT4_G32;
+  const size_t red = gemv_red_bytes(nm, mt, tma_groups(fmt, nm));
   const int nch = klen / (i4 ? 32 : 16);
   const int cbytes = i4 ? Codes<FMT_INT4_G32>::kStageBytes : Codes<FMT_INT8_ROW>::kStageBytes;
   const int tok_rows = (stage_tokens + mt - 1) / mt * mt;
   const size_t x_bytes = ((size_t)tok_rows * ((size_t)nch * cbytes + 4 * nch + (i4 ? 4 * nch : 0)) + 127) / 128 * 128;
-  return 128 + x_bytes + tma_gemv_stage_bytes(fmt, nm, klen) * stages;
+  return 128 + x_bytes + red + tma_gemv_stage_bytes(fmt, nm, klen) * stages;
 }
 
 size_t tma_gemv_stage_bytes(int fmt, int nm, int klen) {

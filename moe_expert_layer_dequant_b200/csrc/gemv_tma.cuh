@@ -11,7 +11,12 @@ constexpr int kTmaConsumers = 8;  // consumer warps per group = rows per stage
 // down projection; more warps to hide the per-stage arithmetic latency), two
 // otherwise (the fused gate/up pair's larger stages leave room for fewer slots,
 // and the INT8 consumers need more registers than 800 threads allow).
-constexpr int tma_groups(int fmt, int nm) { return (nm == 1 && fmt == FMT_INT4_G32) ? 3 : 2; }
+constexpr int tma_groups(int fmt, int nm) { return (void)fmt, (void)nm, 2; }
+// Shared memory of the consumer groups' row-sum exchange: per group two
+// buffers of [warps][rows * matrices * token rows] floats (128-byte granule).
+__host__ __device__ constexpr size_t gemv_red_bytes(int nm, int mt, int groups) {
+  return ((size_t)groups * 2 * kTmaConsumers * kTmaConsumers * nm * mt * 4 + 127) / 128 * 128;
+}
 
 // Tensor maps of one K-split matrix: codes (u64 elements), scales, mins (u16).
 struct QWMaps {
@@ -50,10 +55,17 @@ struct TmaGemvArgs {
   int* tile_cnt;               // down, dense mode: arrivals of the K splits per CTA row range
   uint16_t* res;               // down, dense mode: residual [M][N], updated in place by the last K split
                                // of each row range (null: fp32 partials only, a tail kernel adds them)
+  const uint16_t* norm_w;      // dense gate/up, unsplit K: normalize x on staging (RMSNorm weight [K]), or null
+  float eps;
   int ks_len;                  // K elements per split (INT4: multiple of 256)
   int ctas_per_job;
   int stage_tokens;
   int stages;
+  // Failure-detection tests only (0 in every product launch): the producer
+  // issues no stage from index inject_stop - 1 on, as if it had died, and the
+  // pipeline waits give up after wait_ns (0: the default of about a second).
+  int inject_stop;
+  unsigned long long wait_ns;
 };
 
 // Encodes the three maps of W[N][K] for boxes of [rows_per_stage][ks_len].

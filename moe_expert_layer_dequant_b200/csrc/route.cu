@@ -11,6 +11,7 @@
 #include <algorithm>
 
 #include "launch.cuh"
+#include "norm.cuh"
 #include "route.cuh"
 
 namespace moeffn {
@@ -23,22 +24,47 @@ constexpr int kRouterThreads = 128;
 // row e == E is the shared expert gate vector (bf16), written to gate_logit[t].
 __global__ void __launch_bounds__(kRouterThreads) k_router_logits(const RouterArgs a) {
   __shared__ float red[kRouterThreads / 32];
+  __shared__ float s_inv;
   pdl_launch_dependents();
   pdl_wait();
   const int t = blockIdx.x;
   const int e = blockIdx.y;
   const bool gate_row = (e == a.E);
   const uint16_t* x = a.x + (size_t)t * a.H;
+  const bool norm = a.norm_w != nullptr;
+  float inv = 0.f;
+  if (norm) {
+    // Input norm folded in: every CTA of the token finds the row's inv_rms
+    // (the row is a few KB); the CTA of expert 0 also stores m.
+    float ss = warp_sum(row_sumsq_part(x, a.H, threadIdx.x, kRouterThreads));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float v = 0.f;
+      for (int i = 0; i < kRouterThreads / 32; ++i) v += red[i];   // fixed order
+      s_inv = inv_rms_of(v, a.H, a.eps);
+    }
+    __syncthreads();
+    inv = s_inv;
+    if (e == 0)
+      for (int k = threadIdx.x; k < a.H; k += kRouterThreads)
+        a.m_out[(size_t)t * a.H + k] = prenorm_elem(x[k], a.norm_w[k], inv);
+  }
+  // The token row's k-th value as the layer's input m (normalized or given).
+  auto xval = [&](uint32_t bits16, int k) -> float {
+    return norm ? bf16_bits_to_float(prenorm_elem((uint16_t)bits16, a.norm_w[k], inv))
+                : bf16_bits_to_float((uint16_t)bits16);
+  };
   float acc = 0.f;
   if (!gate_row && a.router_f32) {
     const float* w = reinterpret_cast<const float*>(a.router) + (size_t)e * a.H;
     for (int k = threadIdx.x * 4; k < a.H; k += kRouterThreads * 4) {
       const float4 wv = *reinterpret_cast<const float4*>(w + k);
       const uint2 xv = *reinterpret_cast<const uint2*>(x + k);
-      acc = fmaf(wv.x, __uint_as_float(xv.x << 16), acc);
-      acc = fmaf(wv.y, __uint_as_float(xv.x & 0xFFFF0000u), acc);
-      acc = fmaf(wv.z, __uint_as_float(xv.y << 16), acc);
-      acc = fmaf(wv.w, __uint_as_float(xv.y & 0xFFFF0000u), acc);
+      acc = fmaf(wv.x, xval(xv.x & 0xFFFFu, k), acc);
+      acc = fmaf(wv.y, xval(xv.x >> 16, k + 1), acc);
+      acc = fmaf(wv.z, xval(xv.y & 0xFFFFu, k + 2), acc);
+      acc = fmaf(wv.w, xval(xv.y >> 16, k + 3), acc);
     }
   } else {
     const uint16_t* w = gate_row ? a.w_sg : reinterpret_cast<const uint16_t*>(a.router) + (size_t)e * a.H;
@@ -48,12 +74,13 @@ __global__ void __launch_bounds__(kRouterThreads) k_router_logits(const RouterAr
       const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w}, xx[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        acc = fmaf(__uint_as_float(ww[j] << 16), __uint_as_float(xx[j] << 16), acc);
-        acc = fmaf(__uint_as_float(ww[j] & 0xFFFF0000u), __uint_as_float(xx[j] & 0xFFFF0000u), acc);
+        acc = fmaf(__uint_as_float(ww[j] << 16), xval(xx[j] & 0xFFFFu, k + 2 * j), acc);
+        acc = fmaf(__uint_as_float(ww[j] & 0xFFFF0000u), xval(xx[j] >> 16, k + 2 * j + 1), acc);
       }
     }
   }
   acc = warp_sum(acc);
+  __syncthreads();   // red is reused
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -64,6 +91,27 @@ __global__ void __launch_bounds__(kRouterThreads) k_router_logits(const RouterAr
   }
 }
 
+// m = rms_norm(x, w) of one row per CTA.
+__global__ void __launch_bounds__(256) k_prenorm_rows(const PrenormArgs a) {
+  __shared__ float red[8];
+  __shared__ float s_inv;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int t = blockIdx.x;
+  const uint16_t* x = a.x + (size_t)t * a.H;
+  const float ss = warp_sum(row_sumsq_part(x, a.H, threadIdx.x, 256));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float v = 0.f;
+    for (int i = 0; i < 8; ++i) v += red[i];   // fixed order
+    s_inv = inv_rms_of(v, a.H, a.eps);
+  }
+  __syncthreads();
+  const float inv = s_inv;
+  for (int k = threadIdx.x; k < a.H; k += 256) a.m[(size_t)t * a.H + k] = prenorm_elem(x[k], a.w[k], inv);
+}
+
 // (value, index) order of the top-k: larger value first, lower index on ties.
 __device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
@@ -72,7 +120,7 @@ __device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
 // Top-k of one token by one warp: every lane holds up to PL logits (experts
 // lane, lane+32, ...); k rounds of a warp-wide arg-max, the winner's lane
 // retires it. Weights: softmax over the k selected logits times the
-// per-expert scale (ones), rounded to fp16.
+// per-expert scale of the selected expert (ones unless given), rounded to fp16.
 template <int PL>
 __device__ __forceinline__ void topk_token(const RouteArgs& a, int t, int lane) {
   const float* l = a.logits + (size_t)t * a.E;
@@ -112,7 +160,8 @@ __device__ __forceinline__ void topk_token(const RouteArgs& a, int t, int lane) 
   if (lane == 0) {
     for (int r = 0; r < a.k; ++r) {
       a.idx[t * a.k + r] = ir[r];
-      a.w[t * a.k + r] = __half2float(__float2half_rn(zr[r] / zsum));
+      const float sc = a.scale != nullptr ? a.scale[ir[r]] : 1.0f;
+      a.w[t * a.k + r] = __half2float(__float2half_rn(zr[r] / zsum * sc));
     }
   }
 }
@@ -183,6 +232,10 @@ __global__ void __launch_bounds__(128) k_gather_rows(const GatherArgs a) {
 }
 
 }  // namespace
+
+cudaError_t launch_prenorm_rows(const PrenormArgs& a, cudaStream_t s) {
+  return launch_pdl(k_prenorm_rows, dim3(a.M), dim3(256), 0, s, a);
+}
 
 cudaError_t launch_gather_rows(const GatherArgs& a, cudaStream_t s) {
   return launch_pdl(k_gather_rows, dim3(a.P), dim3(128), 0, s, a);

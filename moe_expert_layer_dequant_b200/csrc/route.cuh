@@ -15,7 +15,22 @@ struct RouterArgs {
   int M, H, E;
   float* logits;               // [M][E]
   float* gate_logit;           // [M] (when w_sg != null)
+  // Input norm folded in: x is the residual; the logits use m = rms_norm(x,
+  // norm_w), which the (token, 0) CTAs also write to m_out [M][H]. Null: x is m.
+  const uint16_t* norm_w;
+  float eps;
+  uint16_t* m_out;
 };
+
+// m = rms_norm(x, w) row by row into m [M][H] (one CTA per row).
+struct PrenormArgs {
+  const uint16_t* x;
+  const uint16_t* w;
+  float eps;
+  int M, H;
+  uint16_t* m;
+};
+cudaError_t launch_prenorm_rows(const PrenormArgs& a, cudaStream_t s);
 
 struct RouteArgs {
   const float* logits;         // [M][E]
@@ -27,6 +42,7 @@ struct RouteArgs {
   int* offsets;                // [E+1]
   int* union_list;             // [E] or null
   int* n_union;                // [1] or null
+  const float* scale;          // [E] per-expert scale of the routing weights, or null (ones)
 };
 
 // xg[s][:] = x[perm[s] / topk][:] for the P = M*topk pair slots (bf16 rows of H).

@@ -14,6 +14,12 @@
 //               seeded with the gated shared expert; no norm in the tail).
 //               seed = bf16(bf16(s) * sigmoid(gate_logit)) with s the shared
 //               expert's down output, or 0 without a shared expert.
+//  * moe, Gemma form: the routed sum starts from 0; the shared branch joins
+//               after its post-FFN norm: h1 = bf16(RMSNorm(bf16(s)) * w),
+//               x = bf16(x + bf16(y + h1)) (turbospark-runtime 0.3.0,
+//               src/families/qwen/moe_batch.rs, module doc on Gemma; the
+//               branch norm of turbospark-runtime 0.1.0,
+//               src/families/gemma4/shared_expert.rs).
 #include "launch.cuh"
 #include "tail.cuh"
 
@@ -81,9 +87,50 @@ __global__ void __launch_bounds__(512) k_tail_rmsnorm(const TailArgs a) {
   }
 }
 
+// Gemma-form MoE tail, one CTA per token row: the shared branch's RMSNorm
+// needs the whole row of its output first.
+__global__ void __launch_bounds__(512) k_tail_moe_gemma(const TailArgs a) {
+  __shared__ float red[16];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int t = blockIdx.x;
+  const size_t sstride = (size_t)a.M * a.N;
+  float ss = 0.f;
+  for (int n = threadIdx.x; n < a.N; n += blockDim.x) {
+    const float h = round_bf16(sum_splits(a.d_s, a.splits_s, sstride, (size_t)t * a.N + n));
+    ss = fmaf(h, h, ss);
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float inv_rms = 1.0f / sqrtf(red[0] / (float)a.N + a.eps);
+  for (int n = threadIdx.x; n < a.N; n += blockDim.x) {
+    const size_t o = (size_t)t * a.N + n;
+    const float h = round_bf16(sum_splits(a.d_s, a.splits_s, sstride, o));
+    const float h1 = round_bf16(h * inv_rms * bf16_bits_to_float(a.norm_w[n]));
+    float acc = 0.f;   // the routed sum starts from nothing
+    for (int r = 0; r < a.k; ++r) {
+      const int slot = a.inv[t * a.k + r];
+      const float dr = sum_splits(a.d, a.splits, (size_t)a.slots * a.N, (size_t)slot * a.N + n);
+      acc = __fadd_rn(acc, __fmul_rn(a.w[t * a.k + r], dr));
+    }
+    const float y = round_bf16(acc);
+    a.res[o] = float_to_bf16_bits(bf16_bits_to_float(a.res[o]) + round_bf16(y + h1));
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_tail(const TailArgs& a, cudaStream_t s) {
+  if (a.mode == TAIL_MOE_GEMMA) {
+    return launch_pdl(k_tail_moe_gemma, dim3(a.M), dim3(512), 0, s, a);
+  }
   if (a.mode == TAIL_RMSNORM) {
     return launch_pdl(k_tail_rmsnorm, dim3(a.M), dim3(512), 16 * sizeof(float), s, a);
   } else {

@@ -4,7 +4,7 @@
 
 namespace moeffn {
 
-enum : int { TAIL_RESIDUAL = 0, TAIL_RMSNORM = 1, TAIL_MOE = 2 };
+enum : int { TAIL_RESIDUAL = 0, TAIL_RMSNORM = 1, TAIL_MOE = 2, TAIL_MOE_GEMMA = 3 };
 
 struct TailArgs {
   int mode;
@@ -19,7 +19,7 @@ struct TailArgs {
   int k;
   uint16_t* res;               // [M][N] residual stream, updated in place
   uint16_t* h1;                // [M][N] RMSNorm output
-  const uint16_t* norm_w;      // [N]
+  const uint16_t* norm_w;      // [N] (RMSNORM: the branch's norm; MOE_GEMMA: the shared branch's post-norm)
   float eps;
 };
 

@@ -317,6 +317,24 @@ def seeded_rank_sum(seed: np.ndarray, w: np.ndarray, d: np.ndarray) -> np.ndarra
     return bf16(acc)
 
 
+def gemma_shared_branch(shared, x_bits: np.ndarray, norm_w_bits: np.ndarray, act: str, eps: float) -> np.ndarray:
+    """The Gemma shared branch that joins the routed layer's tail: the shared
+    FFN, then ``post_feedforward_layernorm_1`` ([gemma]
+    ``encode_shared_expert_branch``: h1 = RMSNorm of the 2-byte down output,
+    in place). Returns float64 [M][H] (bf16 values)."""
+    return bf16_to_f64(ffn_shared_expert(shared, x_bits, norm_w_bits, act, eps))
+
+
+def gemma_routed_tail(res: np.ndarray, y: np.ndarray, h1: np.ndarray) -> np.ndarray:
+    """Tail of the Gemma-style routed layer ([qwen] module doc, contrasting the
+    families: Gemma's "routed sum starts from nothing and its shared branch
+    joins in the sandwich tail after a norm"): the routed output y (summed from
+    zero) and the normed shared branch h1 join as two 2-byte rows, then the
+    raw residual add. Reading: the pages name no other norm for this tail.
+    Returns float64 (bf16 values)."""
+    return bf16(res + bf16(y + h1))
+
+
 def moe_layer(inp, return_internals: bool = False, tokens: Optional[Sequence[int]] = None):
     """Routed MoE layer with optional gated shared expert, raw residual tail.
 
@@ -335,10 +353,11 @@ def moe_layer(inp, return_internals: bool = False, tokens: Optional[Sequence[int
     x = bf16_to_f64(x_bits)
 
     logits = router_logits(inp.router, x_bits)
-    idx, w = topk_softmax(logits, k)
+    gemma = getattr(inp, "shared_norm_w", None) is not None
+    idx, w = topk_softmax(logits, k, getattr(inp, "expert_scale", None))
     perm, offsets, union = expert_permutation(idx, c.E)
 
-    if inp.shared is not None:
+    if inp.shared is not None and not gemma:
         seed = shared_seed(inp.shared, inp.w_sg, x_bits, c.act)
     else:
         seed = np.zeros((M, H))   # the routed sum starts from nothing
@@ -351,11 +370,16 @@ def moe_layer(inp, return_internals: bool = False, tokens: Optional[Sequence[int
         a = gate_up_act(dequant(ex.gate), dequant(ex.up), x[t], c.act)   # phase 1
         d[t, r, :] = a @ dequant(ex.down).T                               # phase 2 (down)
     y = seeded_rank_sum(seed, w, d)
-    out = bf16_bits(residual_add(bf16_to_f64(res_bits), y))
+    h1 = None
+    if gemma:
+        h1 = gemma_shared_branch(inp.shared, x_bits, inp.shared_norm_w, c.act, inp.shared_norm_eps)
+        out = bf16_bits(gemma_routed_tail(bf16_to_f64(res_bits), y, h1))
+    else:
+        out = bf16_bits(residual_add(bf16_to_f64(res_bits), y))
     if not return_internals:
         return out
     return out, dict(logits=logits, idx=idx, w=w, perm=perm, offsets=offsets, union=union,
-                     seed=seed, y=y, d=d)
+                     seed=seed, y=y, d=d, h1=h1)
 
 
 def dense_layer(inp) -> np.ndarray:

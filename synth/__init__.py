@@ -153,6 +153,12 @@ class LayerInputs:
     experts: List[FFNWeights] = field(default_factory=list)
     shared: Optional[FFNWeights] = None
     w_sg: Optional[np.ndarray] = None      # bf16 bits [H]
+    # Gemma-style routed layer: learned per-expert scale of the routing
+    # weights (fp32 [E]; None = ones) and the shared branch's post-FFN norm
+    # weight (bf16 bits [H]; None = the shared expert is gated and seeds the sum)
+    expert_scale: Optional[np.ndarray] = None
+    shared_norm_w: Optional[np.ndarray] = None
+    shared_norm_eps: float = 1e-6
 
     def weight_bytes_total(self) -> int:
         n = 0
@@ -161,7 +167,7 @@ class LayerInputs:
         n += sum(e.nbytes for e in self.experts)
         if self.shared is not None:
             n += self.shared.nbytes
-        for a in (self.norm_w, self.router, self.w_sg):
+        for a in (self.norm_w, self.router, self.w_sg, self.expert_scale, self.shared_norm_w):
             if a is not None:
                 n += a.nbytes
         return n
@@ -204,3 +210,18 @@ def zero_like_qweight(fmt: str, N: int, K: int) -> QWeight:
         return QWeight(fmt, N, K, np.zeros((N, K), np.int8), np.zeros(N, np.float16))
     return QWeight(fmt, N, K, np.zeros((N, K // 2), np.uint8), np.zeros((N, K // 32), np.float16),
                    np.zeros((N, K // 32), np.float16))
+
+
+_T_EXPERT_SCALE, _T_SHARED_NORM = 5, 6
+
+
+def make_gemma_form(li: LayerInputs, seed: int) -> LayerInputs:
+    """The same routed layer in the Gemma form: a per-expert routing scale
+    ~ U(0.5, 2) (fp32) and a post-FFN norm weight of the shared branch
+    ~ 1 + N(0, 0.1) (bf16); the shared gate vector is dropped."""
+    c = li.config
+    out = replace(li)
+    out.expert_scale = _rng(c.cfg, seed, _T_EXPERT_SCALE).uniform(0.5, 2.0, c.E).astype(np.float32)
+    out.shared_norm_w = to_bf16_bits(1.0 + _rng(c.cfg, seed, _T_SHARED_NORM).normal(0.0, 0.1, c.H))
+    out.w_sg = None
+    return out

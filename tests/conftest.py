@@ -30,3 +30,23 @@ def read_golden(name):
             else:
                 rows.append(line.split())
     return kv, rows
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Report how many bf16 rounding flips the output comparisons accepted."""
+    try:
+        import devutil
+    except Exception:
+        return
+    log = getattr(devutil, "FLIP_LOG", [])
+    if not log:
+        return
+    n = sum(e[1] for e in log)
+    flips = sum(e[2] for e in log)
+    with_flips = [e for e in log if e[2]]
+    worst = max(e[3] for e in log)
+    terminalreporter.write_line(
+        f"bf16 output comparisons: {len(log)} calls, {n} elements, {flips} rounding flips accepted "
+        f"(<= 2 bf16 ulps each) in {len(with_flips)} calls; worst other |err| = {worst:.3e} x RMS")
+    for what, size, f, w in sorted(with_flips, key=lambda e: -e[2] / e[1])[:10]:
+        terminalreporter.write_line(f"  {what}: {f} of {size} elements")

@@ -95,3 +95,17 @@ def rank_pairing_layer(H=32, reps=1):
     router[1, 1] = np.float32(math.log(3.0))
     x = _one_hot_rows(H, [0, 1], reps)
     return synth.LayerInputs(c, x.shape[0], 0, x, np.zeros_like(x), router=router, experts=[e0, e1])
+
+
+def gemma_routed_layer(H=256, reps=1):
+    """The Gemma-style routed layer (golden gemma_routed_layer.txt): the routed
+    part of rank_pairing_layer with per-expert scale (2, 0.5), and a shared
+    expert with output 2 at feature 0, post-norm weight ones, residual 0."""
+    li = rank_pairing_layer(H, reps)
+    c = synth.scaled_config(5, H=H, I=H, E=2, k=2, I_s=H, router="f32")
+    li.config = c
+    li.shared = _ffn(H, H, [0, 1], 1, 2.0, 0.0)             # s_0 = 2 for tokens e_0, e_1
+    li.expert_scale = np.array([2.0, 0.5], np.float32)
+    li.shared_norm_w = synth.to_bf16_bits(np.ones(H))
+    li.shared_norm_eps = 1e-6
+    return li

@@ -111,3 +111,14 @@ def test_router_and_plan_refusals():
     desc.top_k = 0
     assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -2
     assert L.moe_layer(None, x, 0x50000000, 1, None, ws, 1 << 20, None) == -1
+
+
+def test_fault_injection_export_validates_on_the_host():
+    """The failure-injection test export refuses unknown kinds, depths outside
+    1..8 and wait limits outside 1 us..1 s before any launch (host only)."""
+    import moe_expert_layer_dequant_b200 as lib
+    for args in ((3, 0, 10), (2, 9, 10), (2, 0, 10), (1, -1, 10), (1, 0, 0), (1, 0, 2000000)):
+        with pytest.raises(lib.MoeffnError) as e:
+            lib.test_inject_gemv_fault(*args)
+        assert e.value.status == -1
+    lib.test_inject_gemv_fault(0)                  # cancel: always accepted

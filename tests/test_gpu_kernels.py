@@ -123,6 +123,30 @@ def test_dense_small(cfg, shape, fmt, M):
     assert_bf16_close(dl.run(inp.x, zero), oracle.layer(inp), "h")
 
 
+@pytest.mark.parametrize("cfg,shape", [(2, dict(H=512, I=1024)), (1, dict(H=512, I=512))])
+@pytest.mark.parametrize("frac", [1.0, 0.125])
+@pytest.mark.parametrize("M", [1, 2])
+def test_decode_gemv_activation_outliers(cfg, shape, frac, M):
+    """The decode GEMV stages activations as int16 with one power-of-two factor
+    per chunk: values far below the chunk's largest lose low bits. Outlier
+    channels are the method's numeric edge case: every chunk (frac 1) or one
+    in eight holds one value of +-2^8 among values of about 2^-6. Residual 0,
+    so the output is bf16(h), checked at the plain tolerance."""
+    c = synth.scaled_config(cfg, **shape)
+    inp = synth.make_inputs(c, M, 6)
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((M, c.H)) * 2.0 ** -6
+    chunk = 32 if c.fmt == FMT_INT4_G32 else 16
+    for t in range(M):
+        for ch in range(c.H // chunk):
+            if rng.random() < frac:
+                x[t, ch * chunk + rng.integers(chunk)] = rng.choice([-1.0, 1.0]) * 256.0
+    inp.x = synth.to_bf16_bits(x)
+    inp.residual = np.zeros_like(inp.residual)
+    dl = DeviceLayer(inp)
+    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), f"h with outliers ({frac})")
+
+
 # Token counts from 3 up run the tensor-core GEMM (tcgen05) where K allows:
 # token tiles of 16..256, several tiles and a ragged last tile.
 DENSE_TC = [
@@ -178,6 +202,54 @@ def test_moe_small(shape, M):
     dl.close()
 
 
+# --------------------------------------------------------------------------- input norm folded in
+
+
+def _norm_w(H, seed):
+    return synth.to_bf16_bits(1.0 + np.random.default_rng(seed).normal(0.0, 0.1, H))
+
+
+PRENORM_DENSE = [
+    (2, dict(H=512, I=1024)),      # INT4: GEMV staging folds the norm (M <= 5), a norm launch before the GEMMs
+    (1, dict(H=256, I=416)),       # INT8
+    (2, dict(H=640, I=1056)),      # K % 256 != 0: register-load GEMV after a norm launch
+]
+
+
+@pytest.mark.parametrize("cfg,shape", PRENORM_DENSE)
+@pytest.mark.parametrize("M", [1, 2, 5, 16, 40])
+def test_dense_prenorm(cfg, shape, M):
+    c = synth.scaled_config(cfg, **shape)
+    inp = synth.make_inputs(c, M, 4)
+    w = _norm_w(c.H, 4)
+    dl = DeviceLayer(inp)
+    res = dev_bf16(inp.residual)
+    lib.ffn_dense_prenorm(dl.ffn, dev_bf16(w), res, c.act, 1e-6)
+    assert_bf16_close(host_bf16(res), oracle.layer_prenorm(inp, w, 1e-6), "out")
+
+
+@pytest.mark.parametrize("shape", [dict(cfg=4, H=256, I=256, E=16, k=4, I_s=256),
+                                   dict(cfg=5, H=512, I=512, E=8, k=2, I_s=0)])
+@pytest.mark.parametrize("M", [1, 3, 9, 40])
+def test_moe_prenorm(shape, M):
+    shape = dict(shape)
+    c = synth.scaled_config(shape.pop("cfg"), **shape)
+    inp = synth.make_inputs(c, M, 5)
+    w = _norm_w(c.H, 5)
+    dl = DeviceLayer(inp)
+    res = dev_bf16(inp.residual)
+    idx = torch.empty((M, c.k), dtype=torch.int32, device="cuda")
+    lib.moe_layer_prenorm(dl.plan, dev_bf16(w), res, 1e-6, idx)
+    from copy import copy
+    normed = copy(inp)
+    normed.x = oracle.rms_norm_prologue(inp.residual, w, 1e-6)
+    ref, it = oracle.moe_layer(normed, return_internals=True)
+    assert np.array_equal(idx.cpu().numpy(), it["idx"])
+    assert_bf16_close(host_bf16(res), ref, "out")
+    assert np.array_equal(ref, oracle.layer_prenorm(inp, w, 1e-6))
+    dl.close()
+
+
 # --------------------------------------------------------------------------- pinned edge cases
 
 
@@ -225,6 +297,35 @@ def test_rank_weights_meet_their_own_expert_outputs_on_gpu(H, reps):
     want = np.tile([float(t) for t in kv["y_feature0"]], reps)
     assert np.array_equal(oracle.bf16_to_f64(out)[:, 0], want)
     assert np.array_equal(out, oracle.layer(li))
+    dl.close()
+
+
+@pytest.mark.parametrize("H,reps", HANDBUILT_PATHS)
+def test_gemma_routed_layer_on_gpu(H, reps):
+    """Gemma form: scale by expert, routed sum from zero, normed shared branch
+    joined in the tail (golden gemma_routed_layer.txt)."""
+    kv, _ = read_golden("gemma_routed_layer.txt")
+    li = handbuilt.gemma_routed_layer(H, reps)
+    dl = DeviceLayer(li)
+    out = dl.run(li.x, li.residual)
+    want = np.tile([float(t) for t in kv["out_feature0"]], reps)
+    assert np.array_equal(oracle.bf16_to_f64(out)[:, 0], want)
+    assert np.array_equal(out, oracle.layer(li))
+    dl.close()
+
+
+@pytest.mark.parametrize("shape", [dict(cfg=4, H=256, I=256, E=16, k=4, I_s=256),
+                                   dict(cfg=5, H=512, I=512, E=8, k=2, I_s=512)])
+@pytest.mark.parametrize("M", [1, 3, 9, 40])
+def test_gemma_form_moe(shape, M):
+    shape = dict(shape)
+    c = synth.scaled_config(shape.pop("cfg"), **shape)
+    inp = synth.make_gemma_form(synth.make_inputs(c, M, 6), 6)
+    dl = DeviceLayer(inp)
+    out, idx = dl.run(inp.x, inp.residual, topk_out=True)
+    ref, it = oracle.moe_layer(inp, return_internals=True)
+    assert np.array_equal(idx, it["idx"])
+    assert_bf16_close(out, ref, "out")
     dl.close()
 
 

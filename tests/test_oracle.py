@@ -438,3 +438,34 @@ def test_prenorm_layer_feeds_the_normed_residual():
     m = oracle.rms_norm_prologue(inp.residual, w, 1e-6)
     want = oracle.ffn_dense(inp.ffn, m, inp.residual, "silu")
     assert np.array_equal(got, want)
+
+
+
+# --------------------------------------------------------------------------- Gemma-style routed layer
+
+
+def test_gemma_routed_layer_golden():
+    """Per-expert scale looked up by expert, routed sum from zero, normed shared
+    branch joined in the tail (golden gemma_routed_layer.txt)."""
+    kv, _ = read_golden("gemma_routed_layer.txt")
+    li = handbuilt.gemma_routed_layer()
+    out, it = oracle.moe_layer(li, return_internals=True)
+    assert list(it["w"][0]) == [float(t) for t in kv["weights_token0"]]
+    assert list(it["w"][1]) == [float(t) for t in kv["weights_token1"]]
+    assert not np.any(it["seed"])                                     # the routed sum starts from nothing
+    assert list(it["y"][:, 0]) == [float(t) for t in kv["y_feature0"]]
+    assert list(it["h1"][:, 0]) == [float(t) for t in kv["h1_feature0"]]
+    assert list(oracle.bf16_to_f64(out)[:, 0]) == [float(t) for t in kv["out_feature0"]]
+    assert not np.any(oracle.bf16_to_f64(out)[:, 1:])
+
+
+def test_topk_per_expert_scale_follows_the_expert():
+    """The scale multiplies the softmax weight of the expert it belongs to and
+    does not change which experts are selected."""
+    logits = np.array([[0.0, 2.0, 1.0, -1.0]])
+    scale = np.array([3.0, 0.5, 2.0, 7.0])
+    idx1, w1 = oracle.topk_softmax(logits, 2)
+    idx2, w2 = oracle.topk_softmax(logits, 2, scale)
+    assert list(idx1[0]) == list(idx2[0]) == [1, 2]
+    z = np.exp(np.array([0.0, -1.0]))
+    assert np.array_equal(w2[0], oracle.f16(z / z.sum() * np.array([0.5, 2.0])))

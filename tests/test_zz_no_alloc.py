@@ -10,26 +10,29 @@ import numpy as np
 import pytest
 
 import synth
-from devutil import DeviceLayer, assert_bf16_close, dev_bf16, host_bf16
+from devutil import DeviceLayer, dev_bf16, host_bf16
 
 pytestmark = pytest.mark.gpu
 
 lib = pytest.importorskip("moe_expert_layer_dequant_b200")
 
 
-@pytest.mark.parametrize("cfg,shape", [(2, dict(H=512, I=1280)), (1, dict(H=512, I=1408)),
-                                       (2, dict(H=256, I=4352))])
-def test_noalloc_matches_workspace_entry_twice(cfg, shape):
+# Token counts 3 and 5 run the weight-streaming GEMVs, 16 and 64 the tcgen05
+# GEMMs (their tensor maps then point into the library's array).
+@pytest.mark.parametrize("cfg,shape,Ms", [(2, dict(H=512, I=1280), (3, 5)), (1, dict(H=512, I=1408), (3, 5)),
+                                          (2, dict(H=256, I=4352), (3, 5)), (2, dict(H=512, I=1280), (16, 64))])
+def test_noalloc_matches_workspace_entry_twice(cfg, shape, Ms):
     c = synth.scaled_config(cfg, **shape)
     w = synth.make_weights(c, 3)
     dl = DeviceLayer(synth.make_inputs(c, 1, 3, weights=w))
-    for M, seed in ((3, 11), (5, 12)):          # two calls in a row, different inputs
+    assert lib.workspace_bytes(lib.KIND_DENSE, max(Ms), c.H, c.I) <= lib.NOALLOC_SCRATCH_BYTES
+    for M, seed in zip(Ms, (11, 12)):           # two calls in a row, different inputs
         inp = synth.make_inputs(c, M, seed, weights=w)
         want = dev_bf16(inp.residual)
         lib.ffn_dense(dl.ffn, dev_bf16(inp.x), want, c.act)
         got = dev_bf16(inp.residual)
         lib.ffn_dense_noalloc(dl.ffn, dev_bf16(inp.x), got, c.act)
-        assert_bf16_close(host_bf16(got), host_bf16(want), f"noalloc M={M}")
+        assert np.array_equal(host_bf16(got), host_bf16(want)), f"noalloc M={M}"   # same kernels, same inputs
 
 
 def test_noalloc_refuses_calls_above_its_array():
