@@ -89,8 +89,10 @@ int check_ffn(const moeffn_ffn& f, const char* name, int H, int I) {
   if ((rc = check_qweight(f.gate, (n + ".gate").c_str(), I, H)) != MOEFFN_OK) return rc;
   if ((rc = check_qweight(f.up, (n + ".up").c_str(), I, H)) != MOEFFN_OK) return rc;
   if ((rc = check_qweight(f.down, (n + ".down").c_str(), H, I)) != MOEFFN_OK) return rc;
-  if (f.gate.format != f.up.format || f.gate.format != f.down.format)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: gate/up/down formats differ", name);
+  // Block types are resolved per tensor; gate and up run in one fused kernel
+  // and so share theirs, while down may differ (a mixed file).
+  if (f.gate.format != f.up.format)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: gate and up formats differ", name);
   return MOEFFN_OK;
 }
 
@@ -126,10 +128,15 @@ int down_splits_any(int K) {
 constexpr size_t kTmaSmemBudget = 200 * 1024;
 constexpr size_t kTmaXBudget = 72 * 1024;
 
-// The bulk copies need 16-byte aligned rows of codes and (INT4) of scales/mins.
+// The bulk copies need 16-byte aligned sources, destinations and sizes. A
+// stage is 8 whole rows (rows per CTA are a multiple of 8, and every valid FFN
+// matrix has a multiple of 8 rows), so unsplit INT4 rows need only K % 32 ==
+// 0; a matrix split along K loads its scale and min boxes through 2-D tensor
+// maps, whose row stride (K / 16 bytes) must be a multiple of 16: K % 256 == 0.
 bool tma_ok(const moeffn_qweight& w) {
   if (w.format == MOEFFN_Q_INT8_ROW) return true;
-  return w.cols % 256 == 0 && aligned16(w.scale) && aligned16(w.min);
+  if (w.rows % 8 != 0 || !aligned16(w.scale) || !aligned16(w.min)) return false;
+  return w.cols % 256 == 0 || down_splits(w.cols, MOEFFN_Q_INT4_AFFINE_G32) == 1;
 }
 bool tma_ok(const moeffn_ffn& f) { return tma_ok(f.gate) && tma_ok(f.up) && tma_ok(f.down); }
 
@@ -312,7 +319,8 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
                   cudaStream_t s, int* splits_out, uint16_t* res, bool* tail_done, const uint16_t* norm_w = nullptr,
                   float eps = 0.f) {
   *tail_done = false;
-  const int fmt = f.gate.format;
+  const int fmt = f.gate.format;     // gate and up (one fused kernel)
+  const int dfmt = f.down.format;    // down: its own block type
   int rc;
   if (M >= kTcMinTokens && tc_ok(f) && aligned16(x)) {
     if (norm_w != nullptr) {
@@ -342,7 +350,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
       MOEFFN_CHECK_CUDA(launch_tc_gemm(g, (I + kTcGateUpFeat - 1) / kTcGateUpFeat, 1, 1, s), "gate/up GEMM launch");
     }
     TcGemmArgs d{};
-    d.fmt = fmt;
+    d.fmt = dfmt;
     d.mode = TC_DOWN;
     d.ntile = ntile;
     d.N = H;
@@ -354,10 +362,10 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.rscale0 = static_cast<const __half*>(f.down.scale);
     const int row_tiles = (H + kTcDownRows - 1) / kTcDownRows;
     const int want = (kSMs + row_tiles * tt - 1) / (row_tiles * tt);
-    d.ks_len = tc_down_slice(I, fmt, want, down_splits_any(I));
+    d.ks_len = tc_down_slice(I, dfmt, want, down_splits_any(I));
     const int splits = (I + d.ks_len - 1) / d.ks_len;
     MOEFFN_CHECK_CUDA(encode_tc_x_map(&d.xmap, w.acts, M, I, ntile), "tensor map encode");
-    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&d.w0, fmt, to_qw(f.down), H, I), "tensor map encode");
+    MOEFFN_CHECK_CUDA(encode_tc_weight_maps(&d.w0, dfmt, to_qw(f.down), H, I), "tensor map encode");
     {
       ProfScope ps("down_gemm_tc", s);
       MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, splits, 1, s), "down GEMM launch");
@@ -365,10 +373,10 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     *splits_out = splits;
     return MOEFFN_OK;
   }
-  const int ks = down_slice(I, fmt), splits = down_splits(I, fmt);
+  const int ks = down_slice(I, dfmt), splits = down_splits(I, dfmt);
   *splits_out = splits;
   const TmaGeom gu = tma_geom(fmt, 2, H, M);
-  const TmaGeom dn = tma_geom(fmt, 1, ks, M);
+  const TmaGeom dn = tma_geom(dfmt, 1, ks, M);
   if (tma_ok(f) && gu.ok && dn.ok) {
     TmaGemvArgs g{};
     g.fmt = fmt;
@@ -412,7 +420,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
       MOEFFN_CHECK_CUDA(launch_tma_gemv(g, 2, gu.mt, 1, 1, s), "gate/up launch");
     }
     TmaGemvArgs d{};
-    d.fmt = fmt;
+    d.fmt = dfmt;
     d.a0 = to_qw(f.down);
     d.N = H;
     d.K = I;
@@ -425,7 +433,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.out_d = w.d;
     d.ks_len = ks;
     d.use_maps = splits > 1;
-    if (d.use_maps) MOEFFN_CHECK_CUDA(encode_qw_maps(&d.dmap, fmt, to_qw(f.down), H, I, ks), "tensor map encode");
+    if (d.use_maps) MOEFFN_CHECK_CUDA(encode_qw_maps(&d.dmap, dfmt, to_qw(f.down), H, I, ks), "tensor map encode");
     d.ctas_per_job = std::max(1, kSMs / splits);
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;
@@ -464,7 +472,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     MOEFFN_CHECK_CUDA(launch_gateup(g, (I + g.rows_per_cta - 1) / g.rows_per_cta, 1, mt_for(M), s), "gate/up launch");
   }
   DownArgs d{};
-  d.fmt = fmt;
+  d.fmt = dfmt;
   d.K = I;
   d.N = H;
   d.w = to_qw(f.down);
@@ -474,7 +482,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
   d.d = w.d;
   d.ks_len = ks;
   d.rows_per_cta = rows_per_cta(H * splits);
-  d.stage_tokens = stage_tokens(fmt, d.ks_len, M);
+  d.stage_tokens = stage_tokens(dfmt, d.ks_len, M);
   {
     ProfScope ps("down_gemv", s);
     MOEFFN_CHECK_CUDA(launch_down(d, (H + d.rows_per_cta - 1) / d.rows_per_cta, splits, 1, mt_for(M), s),
@@ -579,7 +587,7 @@ int dense_entry(const char* who, const moeffn_ffn* w, const uint16_t* x, const u
   }
   if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "%s: x/residual not 16-byte aligned", who);
   if (norm_w == nullptr && x == residual) return fail(MOEFFN_ERR_INVALID, "%s: x aliases residual", who);
-  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax || gemv_stage_bytes(w->gate.format, down_slice(I, w->gate.format), 1) > kStageMax)
+  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax || gemv_stage_bytes(w->down.format, down_slice(I, w->down.format), 1) > kStageMax)
     return fail(MOEFFN_ERR_UNSUPPORTED, "%s: hidden size %d too large for the staged GEMV", who, H);
   Carve c{nullptr};
   carve_dense(c, M, H, I);

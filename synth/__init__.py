@@ -131,11 +131,12 @@ def random_qweight(fmt: str, N: int, K: int, rng: np.random.Generator,
     raise ValueError(f"unknown format {fmt}")
 
 
-def random_ffn(fmt: str, H: int, I: int, cfg: int, seed: int, base_id: int) -> FFNWeights:
+def random_ffn(fmt: str, H: int, I: int, cfg: int, seed: int, base_id: int, down_fmt: Optional[str] = None) -> FFNWeights:
+    """gate, up [I][H] in `fmt`; down [H][I] in `down_fmt` (default: the same)."""
     return FFNWeights(
         gate=random_qweight(fmt, I, H, _rng(cfg, seed, base_id + 0)),
         up=random_qweight(fmt, I, H, _rng(cfg, seed, base_id + 1)),
-        down=random_qweight(fmt, H, I, _rng(cfg, seed, base_id + 2)),
+        down=random_qweight(down_fmt or fmt, H, I, _rng(cfg, seed, base_id + 2)),
     )
 
 
@@ -213,6 +214,16 @@ def zero_like_qweight(fmt: str, N: int, K: int) -> QWeight:
 
 
 _T_EXPERT_SCALE, _T_SHARED_NORM = 5, 6
+
+
+def with_down_format(li: LayerInputs, down_fmt: str, seed: int) -> LayerInputs:
+    """A dense layer whose down projection is stored in another block format
+    (per-tensor block types, as in a mixed quantized file)."""
+    c = li.config
+    out = replace(li)
+    out.ffn = FFNWeights(li.ffn.gate, li.ffn.up,
+                         random_qweight(down_fmt, c.H, c.I, _rng(c.cfg, seed, _T_DENSE + 2)))
+    return out
 
 
 def make_gemma_form(li: LayerInputs, seed: int) -> LayerInputs:

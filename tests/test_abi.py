@@ -81,9 +81,11 @@ def test_refusals_before_launch():
     assert L.ffn_dense(ctypes.byref(bad), x, r, 2, 0, ws, 1 << 30, None) == -1
     fmt = _fake_ffn(lib, 9, 256, 512)                                                # unknown format
     assert L.ffn_dense(ctypes.byref(fmt), x, r, 2, 0, ws, 1 << 30, None) == -2
+    # block types are per tensor, but gate and up share one fused kernel
     mixed = _fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256, 512)
-    mixed.down = _fake_qweight(lib, lib.Q_INT8_ROW, 256, 512, 0x30000000)
+    mixed.up = _fake_qweight(lib, lib.Q_INT8_ROW, 512, 256, 0x30000000)
     assert L.ffn_dense(ctypes.byref(mixed), x, r, 2, 0, ws, 1 << 30, None) == -2
+    assert b"gate and up" in L.moeffn_last_error()
     shape = _fake_ffn(lib, lib.Q_INT8_ROW, 256, 512)
     shape.down = _fake_qweight(lib, lib.Q_INT8_ROW, 512, 256, 0x30000000)           # transposed down
     assert L.ffn_dense(ctypes.byref(shape), x, r, 2, 0, ws, 1 << 30, None) == -1
@@ -111,6 +113,18 @@ def test_router_and_plan_refusals():
     desc.top_k = 0
     assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -2
     assert L.moe_layer(None, x, 0x50000000, 1, None, ws, 1 << 20, None) == -1
+    # Gemma form: the shared branch's post-norm needs a shared expert and excludes its gate.
+    experts4 = (lib._FFN * 8)(*[_fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256, 512) for _ in range(8)])
+    shared = _fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256, 512)
+    gate = lib._QWeight(lib.BF16, 1, 256, 0x12000000, None, None)
+    desc = lib._MoeDesc(8, 2, 0, router, experts4, None, None, None, 0x13000000, 1e-6)
+    assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -1
+    desc = lib._MoeDesc(8, 2, 0, router, experts4, ctypes.pointer(shared), ctypes.pointer(gate), None, 0x13000000, 1e-6)
+    assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -1
+    assert b"shared_gate" in L.moeffn_last_error()
+    assert L.moe_layer_prenorm(None, 0x13000000, 1e-6, 0x50000000, 1, None, ws, 1 << 20, None) == -1
+    f = _fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256, 512)
+    assert L.ffn_dense_prenorm(ctypes.byref(f), None, 1e-6, 0x50000000, 2, 0, ws, 1 << 30, None) == -1
 
 
 def test_fault_injection_export_validates_on_the_host():

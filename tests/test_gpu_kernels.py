@@ -105,9 +105,10 @@ def test_router_logits_and_topk_end_to_end():
 
 DENSE_SMALL = [
     (1, dict(H=256, I=416), FMT_INT8_ROW),      # bulk-copy GEMV (INT8 rows)
-    (2, dict(H=640, I=1056), FMT_INT4_G32),     # K % 256 != 0: register-load GEMV
+    (2, dict(H=640, I=1056), FMT_INT4_G32),     # K % 256 != 0, unsplit: bulk-copy GEMV
     (2, dict(H=512, I=1280), FMT_INT4_G32),     # bulk-copy GEMV, ragged CTA row ranges
-    (2, dict(H=256, I=4352), FMT_INT4_G32),     # down split along K: per-row bulk copies
+    (2, dict(H=256, I=4352), FMT_INT4_G32),     # down split along K: 2-D tensor-map boxes
+    (2, dict(H=256, I=4384), FMT_INT4_G32),     # split K with K % 256 != 0: register-load GEMV
 ]
 
 
@@ -145,6 +146,18 @@ def test_decode_gemv_activation_outliers(cfg, shape, frac, M):
     inp.residual = np.zeros_like(inp.residual)
     dl = DeviceLayer(inp)
     assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), f"h with outliers ({frac})")
+
+
+@pytest.mark.parametrize("cfg,shape,down_fmt", [(2, dict(H=512, I=1280), FMT_INT8_ROW),
+                                                (1, dict(H=512, I=1280), FMT_INT4_G32)])
+@pytest.mark.parametrize("M", [1, 3, 16, 40])
+def test_dense_mixed_block_types(cfg, shape, down_fmt, M):
+    """Block types resolved per tensor: the down projection in another format
+    than gate and up (GEMV and tensor-core paths)."""
+    c = synth.scaled_config(cfg, **shape)
+    inp = synth.with_down_format(synth.make_inputs(c, M, 8), down_fmt, 8)
+    dl = DeviceLayer(inp)
+    assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "out")
 
 
 # Token counts from 3 up run the tensor-core GEMM (tcgen05) where K allows:

@@ -139,16 +139,19 @@ def _perm_matrix(n, shift):
 # --------------------------------------------------------------------------- dense FFN
 
 
-@pytest.mark.parametrize("fmt", [FMT_INT8_ROW, FMT_INT4_G32])
-def test_dense_permutation_closed_form(fmt):
+@pytest.mark.parametrize("fmt,down_fmt", [(FMT_INT8_ROW, FMT_INT8_ROW), (FMT_INT4_G32, FMT_INT4_G32),
+                                          (FMT_INT4_G32, FMT_INT8_ROW), (FMT_INT8_ROW, FMT_INT4_G32)])
+def test_dense_permutation_closed_form(fmt, down_fmt):
     """gate = 2 P1, up = Q/2... with non-symmetric permutations: a transposed
-    operand, swapped gate/up or a dropped scale changes which entries meet."""
+    operand, swapped gate/up or a dropped scale changes which entries meet.
+    Mixed block types (down in another format) give the same closed form."""
     n, M = 64, 3
     P1, P2, P3 = _perm_matrix(n, 5), _perm_matrix(n, 0), _perm_matrix(n, 17)
     if fmt == FMT_INT8_ROW:
-        gate, up, down = _int8_matrix(P1, 2.0), _int8_matrix(P2, 0.5), _int8_matrix(P3, 1.0)
+        gate, up = _int8_matrix(P1, 2.0), _int8_matrix(P2, 0.5)
     else:
-        gate, up, down = _int4_matrix(P1, 2.0, 0.0), _int4_matrix(P2, 0.5, 0.0), _int4_matrix(P3, 1.0, 0.0)
+        gate, up = _int4_matrix(P1, 2.0, 0.0), _int4_matrix(P2, 0.5, 0.0)
+    down = _int8_matrix(P3, 1.0) if down_fmt == FMT_INT8_ROW else _int4_matrix(P3, 1.0, 0.0)
     rng = np.random.default_rng(1)
     x = synth.to_bf16_bits(rng.standard_normal((M, n)))
     res = synth.to_bf16_bits(rng.standard_normal((M, n)))
