@@ -239,6 +239,7 @@ struct MoeWS {
   float* d_s;
   uint16_t* xg;      // token rows in pair-slot order (grouped GEMM operand)
   uint16_t* m;       // [M][H] the normed input, when the layer applies its input norm
+  int* cnt;          // [kSMs] arrival counters of phase 2's row ranges (tail folded into phase 2)
 };
 
 // Down-projection K split shared by the routed and the shared expert jobs.
@@ -273,6 +274,7 @@ MoeWS carve_moe(Carve& c, int M, int H, int Ie, int Is, int E, int k) {
   w.d_s = c.take<float>((size_t)sp.shared * M * H);
   w.xg = c.take<uint16_t>(P * H);
   w.m = c.take<uint16_t>((size_t)M * H);
+  w.cnt = c.take<int>(kSMs);
   return w;
 }
 
@@ -401,7 +403,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
       g.zero_n = kSMs;
     }
     if (norm_w != nullptr) {
-      if (gu.tokens <= 8) {            // folded into the staging of the token rows
+      if (gu.tokens <= kGemvNormTokens) {   // folded into the staging of the token rows
         g.norm_w = norm_w;
         g.eps = eps;
       } else {
@@ -957,6 +959,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
   const TmaGeom gu = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, H, max_tok);
   const TmaGeom dn = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 1, sp.ks_len, max_tok);
   int tc_splits_r = splits_r, tc_splits_s = splits_sh;
+  bool tail_done = false;   // the tail ran inside phase 2
   const bool use_tc = p->tc && M >= kTcMinMoeTokens && aligned16(x);
   if (use_tc) {
     // Token rows in pair-slot order feed phase 1's B operand.
@@ -970,7 +973,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     // sized for the mean load per expert plus half again for the routing
     // spread (an expert holds at most M rows).
     const int per_expert = std::max(1, P / std::min(E, P));
-    const int ntile = tc_ntile_for(std::min(M, per_expert + per_expert / 2 + 1));
+    const int ntile = std::min(kTcMaxTok, (std::min(M, per_expert + per_expert / 2 + 1) + 15) & ~15);
     const int tt = (M + ntile - 1) / ntile;
     TcGemmArgs g{};
     g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
@@ -1070,6 +1073,13 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     g.ctas_per_job = std::max(1, kSMs / jobs);
     g.stage_tokens = gu.tokens;
     g.stages = gu.stages;
+    // Qwen form: the seeded rank-ordered tail runs in phase 2's last CTA of
+    // each row range (phase 1 clears the arrival counters).
+    const bool fold_tail = p->shared_post_norm == nullptr;
+    if (fold_tail) {
+      g.zero_cnt = w.cnt;
+      g.zero_n = kSMs;
+    }
     {
       ProfScope ps("phase1_gateup_gemv_tma", s);
       MOEFFN_CHECK_CUDA(launch_tma_gemv(g, 2, gu.mt, 1, jobs, s), "phase-1 launch");
@@ -1103,6 +1113,16 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     d.ctas_per_job = std::max(1, kSMs / (jobs * splits));
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;
+    if (fold_tail) {
+      d.tile_cnt = w.cnt;
+      d.moe_res = residual;
+      d.gate_logit = w.gate_logit;
+      d.route_w = w.w;
+      d.inv = w.inv;
+      d.splits_r = splits_r;
+      d.splits_s = splits_sh;
+      tail_done = true;
+    }
     {
       ProfScope ps("phase2_down_gemv_tma", s);
       MOEFFN_CHECK_CUDA(launch_tma_gemv(d, 1, dn.mt, splits, jobs, s), "phase-2 launch");
@@ -1168,6 +1188,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
   }
   }
 
+  if (tail_done) return MOEFFN_OK;
   TailArgs t{};
   t.mode = p->shared_post_norm != nullptr ? TAIL_MOE_GEMMA : TAIL_MOE;
   t.norm_w = p->shared_post_norm;

@@ -21,15 +21,17 @@
 //              A and B slots with tcgen05.commit;
 //  warp 2      token producer: TMA loads of the bf16 token tiles (128-byte
 //              swizzled, K = 64 per stage), the MMA's B operand;
-//  warps 4-19  dequantize, in two sets of eight taking the K groups in turn:
-//              a thread owns one weight row of one A tile and turns the 32
-//              codes of a quantization group into bf16 (RNE of the exact fp32
-//              value q * scale + min), stored to its TMEM lane (16 columns of
-//              bf16 pairs); then, as the epilogue, read the accumulators
-//              (tcgen05.ld) and write the outputs.
+//  warps 4-19  dequantize, in two sets of eight taking the A stages (K = 64)
+//              in turn: a thread owns one weight row of one A tile and turns
+//              the 64 codes of two quantization groups into bf16 (RNE of the
+//              exact fp32 value q * scale + min), stored to its TMEM lane (32
+//              columns of bf16 pairs); then, as the epilogue, read the
+//              accumulators (tcgen05.ld) and write the outputs.
 //
 // TMEM columns: accumulator of A tile t at [t * ntile, (t + 1) * ntile); a ring
-// of A stages (one K group of 32 each: 16 columns per A tile) after them.
+// of A stages (two K groups each: 32 columns per A tile) after them. Waits
+// suspend the waiting thread (mbarrier.try_wait) rather than spin, so the
+// producer and MMA threads take no issue slots from the dequantizing warps.
 // Modes: GATEUP writes bf16(act(gate) * up); DOWN writes fp32 partial sums
 // d[split][slot][row] that the layer tails combine. INT8-row weights enter the
 // MMA as their exact integer codes and are scaled per row in the epilogue.
@@ -50,7 +52,7 @@ constexpr int kSW = 3;                       // quantized weight stages
 constexpr int kSB = 3;                       // token stages (K = 64 each)
 constexpr int kBStageBytes = kTcMaxTok * 128;
 constexpr int kTmemCols = 512;
-constexpr int kAStageCols = 16 * kTilesA;    // one K group (32 bf16 = 16 columns) per A tile
+constexpr int kAStageCols = 32 * kTilesA;    // two K groups (64 bf16 = 32 columns) per A tile
 
 template <int FMT>
 struct TcFmt;
@@ -210,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   const int k0 = split * a.ks_len;
   if (k0 >= job.K) return;
   const int klen = min(a.ks_len, job.K - k0);     // a multiple of the weight stage K
-  const int nA = klen / 32;                         // A stages (K groups)
+  const int nA = klen / 64;                         // A stages (two K groups each)
   const int nW = klen / F::kKTile;                  // weight stages
   const int nB = klen / 64;                         // token stages
   const int tn = min(ntile, job.ntok - t0);         // valid token rows
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
       int issued = 0;
       for (int w = 0; w < nW; ++w, ++issued) {
         const int slot = w % kSW, use = w / kSW;
-        if (use > 0 && !mbar_wait_spin(&w_empty[slot], (use - 1) & 1)) break;
+        if (use > 0 && !mbar_wait(&w_empty[slot], (use - 1) & 1)) break;
         uint8_t* gst = gbase + (w_base - base) + slot * F::kStageBytes;
         mbar_arrive_expect_tx(&w_full[slot], tx);
         const int kc = k0 + w * F::kKTile;                  // first K element of the stage
@@ -278,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
       }
       // No copy is left in flight when the CTA exits (after a timed-out wait
       // too): the last stages issued have landed.
-      for (int w = max(0, issued - kSW); w < issued; ++w) mbar_wait_spin(&w_full[w % kSW], (w / kSW) & 1);
+      for (int w = max(0, issued - kSW); w < issued; ++w) mbar_wait(&w_full[w % kSW], (w / kSW) & 1);
     }
   } else if (warp == 2) {
     // ---------------- token producer ----------------
@@ -286,34 +288,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
       int issued = 0;
       for (int b = 0; b < nB; ++b, ++issued) {
         const int slot = b % kSB, use = b / kSB;
-        if (use > 0 && !mbar_wait_spin(&b_empty[slot], (use - 1) & 1)) break;
+        if (use > 0 && !mbar_wait(&b_empty[slot], (use - 1) & 1)) break;
         mbar_arrive_expect_tx(&b_full[slot], (uint32_t)ntile * 128u);
         uint8_t* dst = gbase + (b_base - base) + slot * kBStageBytes;
         tma_load_2d(dst, job.xmap, k0 + b * 64, row_tok, &b_full[slot]);
       }
-      for (int b = max(0, issued - kSB); b < issued; ++b) mbar_wait_spin(&b_full[b % kSB], (b / kSB) & 1);
+      for (int b = max(0, issued - kSB); b < issued; ++b) mbar_wait(&b_full[b % kSB], (b / kSB) & 1);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && SA >= 2) {
       const uint32_t idesc = idesc_bf16_f32(kTcRowsA, nmma);
       for (int s = 0; s < nA; ++s) {
-        const int slot = s % SA, bs = (s / 2) % kSB;
-        if (!mbar_wait_spin(&a_full[slot], (s / SA) & 1)) break;
-        if ((s & 1) == 0 && !mbar_wait_spin(&b_full[bs], ((s / 2) / kSB) & 1)) break;
+        const int slot = s % SA, bs = s % kSB;
+        if (!mbar_wait(&a_full[slot], (s / SA) & 1)) break;
+        if (!mbar_wait(&b_full[bs], (s / kSB) & 1)) break;
         tc_fence_after();
-        const uint64_t bd = umma_desc_sw128(b_base + bs * kBStageBytes) + (uint64_t)((s & 1) * 4);
+        const uint64_t bd = umma_desc_sw128(b_base + bs * kBStageBytes);
         const uint32_t acol = tmem + a_col0 + (uint32_t)(slot * kAStageCols);
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk)
+        for (int kk = 0; kk < 4; ++kk)
           for (int t = 0; t < tiles; ++t)
-            umma_bf16_ts(tmem + (uint32_t)(t * ntile), acol + (uint32_t)(t * 16 + kk * 8), bd + 2 * kk, idesc,
+            umma_bf16_ts(tmem + (uint32_t)(t * ntile), acol + (uint32_t)(t * 32 + kk * 8), bd + 2 * kk, idesc,
                          (s | kk) != 0);
         umma_commit(&a_empty[slot]);
-        if (s & 1) umma_commit(&b_empty[bs]);
+        umma_commit(&b_empty[bs]);
       }
       umma_commit(acc_full);
-      mbar_wait_spin(acc_full, 0);   // every MMA has completed before TMEM is freed
+      mbar_wait(acc_full, 0);   // every MMA has completed before TMEM is freed
     }
   } else if (warp >= 4) {
     // ---------------- dequantize (warps 4-19), then epilogue ----------------
@@ -324,24 +326,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
     bool dead = SA < 2;
     for (int s = set; s < nA && !dead; s += 2) {
       const int slot = s % SA, use = s / SA;
-      const int w = s / F::kGroups, g = s % F::kGroups, ws = w % kSW;
+      constexpr int kAPerW = F::kGroups / 2;                           // A stages per weight stage
+      const int w = s / kAPerW, g = 2 * (s % kAPerW), ws = w % kSW;
       bool ok = true;
-      if (g == set) ok = mbar_wait(&w_full[ws], (w / kSW) & 1);          // first group of the stage for this set
+      if (s % kAPerW == set) ok = mbar_wait(&w_full[ws], (w / kSW) & 1);   // first A stage of the weight stage for this set
       if (ok && use > 0) ok = mbar_wait(&a_empty[slot], (use - 1) & 1);
       if (__any_sync(0xffffffffu, !ok)) { dead = true; break; }
       if (t < tiles) {
-        uint32_t o[16];
+        uint32_t o0[16], o1[16];
         const uint32_t tile = w_base + ws * F::kStageBytes + t * F::kTileBytes;
-        if (FMT == FMT_INT4_G32) dq_group_int4(tile, r, g, o);
-        else dq_group_int8(tile, r, g, o);
-        tmem_st16(tmem + lane_base + a_col0 + (uint32_t)(slot * kAStageCols + t * 16), o);
+        if (FMT == FMT_INT4_G32) { dq_group_int4(tile, r, g, o0); dq_group_int4(tile, r, g + 1, o1); }
+        else { dq_group_int8(tile, r, g, o0); dq_group_int8(tile, r, g + 1, o1); }
+        const uint32_t ta = tmem + lane_base + a_col0 + (uint32_t)(slot * kAStageCols + t * 32);
+        tmem_st16(ta, o0);
+        tmem_st16(ta + 16, o1);
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&a_full[slot]);
-        if (g == F::kGroups - 2 + set) mbar_arrive(&w_empty[ws]);   // this set's last group of the stage
+        if (s % kAPerW == kAPerW - 2 + set) mbar_arrive(&w_empty[ws]);   // this set's last A stage of the weight stage
       }
     }
     // Epilogue: TMEM lanes = weight rows, columns = token rows of the tile.

@@ -60,11 +60,6 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
   asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
 }
 
-// Barrier of one consumer group (ids 2.. for the groups).
-__device__ __forceinline__ void group_sync(int grp, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(2 + grp), "r"(nthreads) : "memory");
-}
-
 // NC consumer warps per group, G groups: group g takes the stages s with
 // s % G == g, one row of the stage per warp (R = NC rows per stage). The ring
 // depth S is a multiple of G, so every slot is waited on by one group only,
@@ -118,8 +113,8 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   float* xf = reinterpret_cast<float*>(xi + (size_t)tok_rows * tok_stride);  // [tok_rows][nch] factors
   float* xsum = xf + (size_t)tok_rows * nch;                        // [tok_rows][nch] (INT4)
   const size_t x_bytes = ((size_t)tok_rows * (tok_stride + 4 * nch + (kInt4 ? 4 * nch : 0)) + 127) / 128 * 128;
-  // then the group's row-sum exchange buffers [G][2][NC][R * NM * MT] floats
-  uint8_t* stage0 = smem + 128 + x_bytes + gemv_red_bytes(NM, MT, G);
+  // then the input norm's scratch (gemv_norm_bytes)
+  uint8_t* stage0 = smem + 128 + x_bytes + gemv_norm_bytes(NC * G);
   const size_t stage_bytes = (size_t)NM * R * (cs + 4 * gst);
   // within a stage: codes [NM][R][cs], scales [NM][R][gst], mins [NM][R][gst]
 
@@ -187,40 +182,25 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   }
 
   // ---------------- consumers ----------------
-  // Lane mapping: lane l of a warp owns chunk 32 b + l of the K slice (b a
-  // K block of 32 chunks); the warps of a group split the K blocks and, when
-  // there are fewer K blocks than warps, the stage's rows (row phases: warp
-  // phase j takes rows j, j + P, ...). A lane loads its chunk's staged
-  // activations once per stage and token pass and multiplies them with the
-  // codes of every row it owns; the row sums are then reduced across the
-  // warp (transposed butterfly), across the group's warps through shared
-  // memory (fixed order) and written by one warp per row.
   if (early) pdl_wait();
   const int nthreads = NC * G * 32;
   if (a.zero_cnt != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
     for (int i = threadIdx.x; i < a.zero_n; i += nthreads) a.zero_cnt[i] = 0;
-  const int grp = warp / NC, wr = warp - grp * NC;  // group, warp within the group
+  const int grp = warp / NC, wr = warp - grp * NC;  // group, row of the stage
+  // Shared memory of the input-norm pass: [tok_rows] inverse RMS values, then
+  // [tok_rows][consumer warps] partial sums of squares.
+  float* norm_buf = reinterpret_cast<float*>(smem + 128 + x_bytes);
   const uint16_t* src = job.shared ? a.x_s : a.x;
   const int ld = job.shared ? job.K : a.ld_x;
-  const int nkb = (nch + 31) / 32;                  // K blocks of 32 chunks
-  const int P = nkb >= NC ? 1 : NC / nkb;           // row phases
-  const int wj = P > 1 ? wr / nkb : 0;              // this warp's row phase
-  const int wb = P > 1 ? wr % nkb : wr;             // its first K block
-  const int bstep = P > 1 ? nkb : NC;               // K blocks between its blocks
-  const bool wactive = wj < P;
-  constexpr int V = R * NM * MT;                    // row sums per stage and token pass
-  float* red = reinterpret_cast<float*>(smem + 128 + x_bytes) + (size_t)grp * 2 * NC * V;   // [G][2][NC][V]
-  const int mn_off = NM * R * gst * 2;              // mins follow the scales in a stage
   bool dead = false;
-  int pass = 0;                                     // stage passes of this group (red buffer parity)
   for (int tb = 0, tbi = 0; tb < job.ntok; tb += a.stage_tokens, ++tbi) {
     const int tn = min(a.stage_tokens, job.ntok - tb);
     consumer_sync(nthreads);
     // Input norm folded in (dense gate/up: the job's whole row is this CTA's
     // K range): inv_rms of every staged token row, from per-warp sums of
-    // squares added in warp order. The exchange buffers are free here.
+    // squares added in warp order.
     const bool norm = a.norm_w != nullptr;
-    float* inv_rms = reinterpret_cast<float*>(smem + 128 + x_bytes);   // [tok_rows], then [tok_rows][warps] partial sums
+    float* inv_rms = norm_buf;                        // [tok_rows], then [tok_rows][warps] partial sums
     if (norm) {
       const int nw = nthreads / 32;
       float* ssp = inv_rms + tok_rows;
@@ -255,108 +235,109 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
     for (int rs = grp; rs < row_stages; rs += G) {
       const int s = tbi * row_stages + rs;
       const int slot = s % S, use = s / S;
-      const int n0 = r0 + rs * R;                   // first row of the stage
+      const int n = r0 + rs * R + wr;
+      float row_scale[NM];
+      if (!kInt4 && n < r1) {
+#pragma unroll
+        for (int i = 0; i < NM; ++i) row_scale[i] = __half2float(__ldg(job.m[i].scale + n));
+      }
       // After a timed-out wait (a fault already recorded) the warp stops
       // computing but still takes part in every barrier below.
       if (!dead && !mbar_wait(&full[slot], use & 1, wait_ns)) dead = true;
-      dead = __any_sync(0xffffffffu, dead);
-      const uint8_t* st = stage0 + slot * (int)stage_bytes;
-      for (int tc = 0; tc < tn; tc += MT, ++pass) {
-        float part[V];
+      if (!dead && n < r1) {
+        // 32-bit byte offsets from the stage start (shared memory).
+        const uint8_t* st = stage0 + slot * (int)stage_bytes;
+        int o_code[NM], o_sc[NM];
 #pragma unroll
-        for (int v = 0; v < V; ++v) part[v] = 0.f;
-        if (!dead && wactive) {
-          for (int b = wb; b < nkb; b += bstep) {
-            const int c = 32 * b + lane;
-            if (c >= nch) continue;
-            uint4 x4[MT][C::kChunk / 8];
-            float f[MT], X[MT];
+        for (int i = 0; i < NM; ++i) {
+          o_code[i] = (i * R + wr) * cs + lane * 16;
+          o_sc[i] = NM * R * cs + ((i * R + wr) * gst + lane) * 2;
+        }
+        const int mn_off = NM * R * gst * 2;   // mins follow the scales
+        for (int tc = 0; tc < tn; tc += MT) {
+          float acc[NM][MT];
 #pragma unroll
-            for (int t = 0; t < MT; ++t) {
+          for (int i = 0; i < NM; ++i)
 #pragma unroll
-              for (int q = 0; q < C::kChunk / 8; ++q)
-                x4[t][q] = *reinterpret_cast<const uint4*>(xi + (tc + t) * tok_stride + c * C::kStageBytes + q * 16);
-              f[t] = xf[(tc + t) * nch + c];
-              X[t] = kInt4 ? xsum[(tc + t) * nch + c] : 0.f;
+            for (int t = 0; t < MT; ++t) acc[i][t] = 0.f;
+          int ox = tc * tok_stride + lane * C::kStageBytes;   // staged activations
+          int of = tc * nch + lane;                            // factors / sums
+          int oc = 0, og = 0;                                  // code / scale advance
+          for (int c = lane; c < nch; c += 32, ox += 32 * C::kStageBytes, of += 32, oc += 512, og += 64) {
+            uint4 wv[NM];
+            float sc[NM], mn[NM];
+#pragma unroll
+            for (int i = 0; i < NM; ++i) {
+              wv[i] = *reinterpret_cast<const uint4*>(st + o_code[i] + oc);
+              if (kInt4) {
+                sc[i] = __half2float(*reinterpret_cast<const __half*>(st + o_sc[i] + og));
+                mn[i] = __half2float(*reinterpret_cast<const __half*>(st + o_sc[i] + og + mn_off));
+              }
             }
+            int p0[NM][MT], p1[NM][MT];
 #pragma unroll
-            for (int r = 0; r < R; ++r) {
-              if (r % P != wj) continue;            // rows of this warp's phase
+            for (int i = 0; i < NM; ++i)
 #pragma unroll
-              for (int i = 0; i < NM; ++i) {
-                const uint4 wv = *reinterpret_cast<const uint4*>(st + (size_t)(i * R + r) * cs + c * 16);
-                float sc = 0.f, mn = 0.f;
-                if (kInt4) {
-                  const int o = NM * R * cs + ((i * R + r) * gst + c) * 2;
-                  sc = __half2float(*reinterpret_cast<const __half*>(st + o));
-                  mn = __half2float(*reinterpret_cast<const __half*>(st + o + mn_off));
-                }
+              for (int t = 0; t < MT; ++t) p0[i][t] = p1[i][t] = 0;
+            if (kInt4) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
 #pragma unroll
                 for (int t = 0; t < MT; ++t) {
-                  int p0 = 0, p1 = 0;
-                  if (kInt4) {
-                    Codes<FMT_INT4_G32>::dot_word(wv.x, x4[t][0], p0, p1);
-                    Codes<FMT_INT4_G32>::dot_word(wv.y, x4[t][1 % (C::kChunk / 8)], p0, p1);
-                    Codes<FMT_INT4_G32>::dot_word(wv.z, x4[t][2 % (C::kChunk / 8)], p0, p1);
-                    Codes<FMT_INT4_G32>::dot_word(wv.w, x4[t][3 % (C::kChunk / 8)], p0, p1);
-                  } else {
-                    Codes<FMT_INT8_ROW>::dot_word(wv.x, wv.y, x4[t][0], p0, p1);
-                    Codes<FMT_INT8_ROW>::dot_word(wv.z, wv.w, x4[t][1 % (C::kChunk / 8)], p0, p1);
+                  const uint4 x4 = *reinterpret_cast<const uint4*>(xi + ox + t * tok_stride + q * 16);
+#pragma unroll
+                  for (int i = 0; i < NM; ++i) {
+                    const uint32_t w = q == 0 ? wv[i].x : q == 1 ? wv[i].y : q == 2 ? wv[i].z : wv[i].w;
+                    Codes<FMT_INT4_G32>::dot_word(w, x4, p0[i][t], p1[i][t]);
                   }
-                  const float Pq = (float)(p0 + p1);   // exact below 2^24
-                  // sum_k (q_k s + m) x_k = s * 2^(e-14) * sum_k q_k xi_k + m * sum_k x_k
-                  float& acc = part[(r * NM + i) * MT + t];
-                  acc = kInt4 ? fmaf(sc * f[t], Pq, fmaf(mn, X[t], acc)) : fmaf(f[t], Pq, acc);
+                }
+              }
+            } else {
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                  const uint4 x4 = *reinterpret_cast<const uint4*>(xi + ox + t * tok_stride + h * 16);
+#pragma unroll
+                  for (int i = 0; i < NM; ++i) {
+                    const uint32_t w0 = h == 0 ? wv[i].x : wv[i].z, w1 = h == 0 ? wv[i].y : wv[i].w;
+                    Codes<FMT_INT8_ROW>::dot_word(w0, w1, x4, p0[i][t], p1[i][t]);
+                  }
                 }
               }
             }
-          }
-        }
-        // Warp sums: a transposed butterfly leaves lane l with value
-        // l >> (5 - log2 V) summed over the warp's 32 lanes.
-        int live = V;
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-          if (live > 1) {
-            const bool upper = (lane & o) != 0;
+            for (int t = 0; t < MT; ++t) {
+              const float f = xf[of + t * nch];
+              const float X = kInt4 ? xsum[of + t * nch] : 0.f;
 #pragma unroll
-            for (int k = 0; k < V / 2; ++k) {
-              if (k < live / 2) {
-                const float send = upper ? part[k] : part[k + live / 2];
-                const float keep = upper ? part[k + live / 2] : part[k];
-                part[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+              for (int i = 0; i < NM; ++i) {
+                const float P = (float)(p0[i][t] + p1[i][t]);   // exact below 2^24
+                // sum_k (q_k s + m) x_k = s * 2^(e-14) * sum_k q_k xi_k + m * sum_k x_k
+                acc[i][t] = kInt4 ? fmaf(sc[i] * f, P, fmaf(mn[i], X, acc[i][t])) : fmaf(f, P, acc[i][t]);
               }
             }
-            live >>= 1;
-          } else {
-            part[0] += __shfl_xor_sync(0xffffffffu, part[0], o);
           }
-        }
-        constexpr int kLog2V = V == 8 ? 3 : (V == 16 ? 4 : 5);
-        float* rb = red + (size_t)(pass & 1) * NC * V;
-        if ((lane & ((1 << (5 - kLog2V)) - 1)) == 0) rb[wr * V + (lane >> (5 - kLog2V))] = part[0];
-        group_sync(grp, NC * 32);
-        // Row r of the stage: warp r adds the group's warp sums in warp order.
-        const int n = n0 + wr;
-        if (!dead && n < r1 && lane < NM * MT) {
-          const int i = lane / MT, t = lane % MT;
-          float v = 0.f;
-          for (int w = 0; w < NC; ++w) v += rb[w * V + (wr * NM + i) * MT + t];
-          if (!kInt4) v *= __half2float(__ldg(job.m[i].scale + n));
-          float other = 0.f;   // NM == 2: the up sum of the same token, from lane MT + t
-          if (NM == 2) other = __shfl_down_sync((1u << (NM * MT)) - 1u, v, MT);
-          const int tok = tb + tc + t;
-          if (tok < tn + tb) {
-            const int slot_out = job.slot0 + tok;
-            if (NM == 2) {
-              if (i == 0) {
+          // epilogue
+#pragma unroll
+          for (int t = 0; t < MT; ++t) {
+            float v[NM];
+#pragma unroll
+            for (int i = 0; i < NM; ++i) {
+              v[i] = warp_sum(acc[i][t]);
+              if (!kInt4) v[i] *= row_scale[i];
+            }
+            const int tok = tb + tc + t;
+            if (lane == 0 && tok < tn + tb) {
+              const int slot_out = job.slot0 + tok;
+              if (NM == 2) {
                 uint16_t* out = job.shared ? a.out_act_s : a.out_act;
-                out[(size_t)slot_out * job.N + n] = float_to_bf16_bits(gated_act(v, other, a.act));
+                out[(size_t)slot_out * job.N + n] = float_to_bf16_bits(gated_act(v[0], v[NM - 1], a.act));
+              } else {
+                float* d = job.shared ? a.out_d_s : a.out_d;
+                const int nslots = job.shared ? a.M : a.slots;
+                d[((size_t)blockIdx.y * nslots + slot_out) * job.N + n] = v[0];
               }
-            } else {
-              float* d = job.shared ? a.out_d_s : a.out_d;
-              const int nslots = job.shared ? a.M : a.slots;
-              d[((size_t)blockIdx.y * nslots + slot_out) * job.N + n] = v;
             }
           }
         }
@@ -393,6 +374,46 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
       }
     }
   }
+
+  if (a.moe_res != nullptr) {
+    // MoE tail folded in: every routed expert's and the shared expert's K
+    // splits write this row range; the last of them to finish forms, per
+    // token, seed = bf16(bf16(s) * sigmoid(gate logit)) (0 without a shared
+    // expert), adds w_r * d_r for the ranks r = 0..k-1 in order (fp32) and
+    // adds bf16 of the sum to the residual: the arithmetic of the tail kernel.
+    __threadfence();
+    consumer_sync(nthreads);
+    int* last = reinterpret_cast<int*>(xi);   // staged activations are no longer read
+    if (threadIdx.x == 0) {
+      const int expected = *a.n_union * a.splits_r + (a.Ns > 0 ? a.splits_s : 0);
+      const int old = atomicAdd(&a.tile_cnt[blockIdx.x], 1);
+      *last = old == expected - 1;
+      if (*last) a.tile_cnt[blockIdx.x] = 0;  // ready for the next call
+    }
+    consumer_sync(nthreads);
+    if (*last) {
+      __threadfence();
+      const int nr = r1 - r0, N = job.N;
+      const size_t rstride = (size_t)a.slots * N, sstride = (size_t)a.M * N;
+      for (int i = threadIdx.x; i < nr * a.M; i += nthreads) {
+        const int t = i / nr, n = r0 + (i - t * nr);
+        float acc = 0.f;
+        if (a.Ns > 0) {   // a shared expert seeds the sum
+          float sh = 0.f;
+          for (int sp = 0; sp < a.splits_s; ++sp) sh += __ldcg(a.out_d_s + sp * sstride + (size_t)t * N + n);
+          acc = round_bf16(round_bf16(sh) * sigmoid_f(__ldcg(a.gate_logit + t)));
+        }
+        for (int r = 0; r < a.topk; ++r) {
+          const int slot = __ldcg(a.inv + t * a.topk + r);
+          float dr = 0.f;
+          for (int sp = 0; sp < a.splits_r; ++sp) dr += __ldcg(a.out_d + sp * rstride + (size_t)slot * N + n);
+          acc = __fadd_rn(acc, __fmul_rn(__ldcg(a.route_w + t * a.topk + r), dr));
+        }
+        const size_t o = (size_t)t * N + n;
+        a.moe_res[o] = float_to_bf16_bits(bf16_bits_to_float(a.moe_res[o]) + round_bf16(acc));
+      }
+    }
+  }
 }
 
 template <int FMT, int MT, int NM>
@@ -416,7 +437,7 @@ size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
 
 size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages) {
   const bool i4 = fmt == FMT_INT4_G32;
-  const size_t red = gemv_red_bytes(nm, mt, tma_groups(fmt, nm));
+  const size_t red = gemv_norm_bytes(kTmaConsumers * tma_groups(fmt, nm));
   const int nch = klen / (i4 ? 32 : 16);
   const int cbytes = i4 ? Codes<FMT_INT4_G32>::kStageBytes : Codes<FMT_INT8_ROW>::kStageBytes;
   const int tok_rows = (stage_tokens + mt - 1) / mt * mt;

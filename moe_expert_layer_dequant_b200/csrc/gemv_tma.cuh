@@ -11,11 +11,13 @@ constexpr int kTmaConsumers = 8;  // consumer warps per group = rows per stage
 // down projection; more warps to hide the per-stage arithmetic latency), two
 // otherwise (the fused gate/up pair's larger stages leave room for fewer slots,
 // and the INT8 consumers need more registers than 800 threads allow).
-constexpr int tma_groups(int fmt, int nm) { return (void)fmt, (void)nm, 2; }
-// Shared memory of the consumer groups' row-sum exchange: per group two
-// buffers of [warps][rows * matrices * token rows] floats (128-byte granule).
-__host__ __device__ constexpr size_t gemv_red_bytes(int nm, int mt, int groups) {
-  return ((size_t)groups * 2 * kTmaConsumers * kTmaConsumers * nm * mt * 4 + 127) / 128 * 128;
+constexpr int tma_groups(int fmt, int nm) { return (nm == 1 && fmt == FMT_INT4_G32) ? 3 : 2; }
+// Token rows whose input norm the GEMV's staging applies (more: a norm launch first).
+constexpr int kGemvNormTokens = 8;
+// Shared memory of the staging's input-norm pass: inverse RMS per staged token
+// row and the consumer warps' partial sums of squares (128-byte granule).
+__host__ __device__ constexpr size_t gemv_norm_bytes(int consumer_warps) {
+  return ((size_t)kGemvNormTokens * (1 + consumer_warps) * 4 + 127) / 128 * 128;
 }
 
 // Tensor maps of one K-split matrix: codes (u64 elements), scales, mins (u16).
@@ -55,6 +57,15 @@ struct TmaGemvArgs {
   int* tile_cnt;               // down, dense mode: arrivals of the K splits per CTA row range
   uint16_t* res;               // down, dense mode: residual [M][N], updated in place by the last K split
                                // of each row range (null: fp32 partials only, a tail kernel adds them)
+  // Down, grouped mode (MoE phase 2, Qwen form): the last CTA to finish a row
+  // range, over every routed expert's and the shared expert's jobs and K
+  // splits, adds the seeded rank-ordered sum of that range to moe_res in place
+  // (null: a tail kernel does it). Arrivals are counted in tile_cnt.
+  uint16_t* moe_res;           // [M][N]
+  const float* gate_logit;     // [M] shared-expert gate logits (with a shared expert)
+  const float* route_w;        // [M][k] routing weights
+  const int* inv;              // [M*k] slot of pair p
+  int splits_r, splits_s;      // K splits of the routed and the shared jobs
   const uint16_t* norm_w;      // dense gate/up, unsplit K: normalize x on staging (RMSNorm weight [K]), or null
   float eps;
   int ks_len;                  // K elements per split (INT4: multiple of 256)

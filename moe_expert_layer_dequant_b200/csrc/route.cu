@@ -118,12 +118,12 @@ __device__ __forceinline__ bool beats(float v, int i, float bv, int bi) {
 }
 
 // Top-k of one token by one warp: every lane holds up to PL logits (experts
-// lane, lane+32, ...); k rounds of a warp-wide arg-max, the winner's lane
-// retires it. Weights: softmax over the k selected logits times the
-// per-expert scale of the selected expert (ones unless given), rounded to fp16.
+// lane, lane+32, ...) of the token's row `l`; k rounds of a warp-wide
+// arg-max, the winner's lane retires it. Weights: softmax over the k selected
+// logits times the per-expert scale of the selected expert (ones unless
+// given), rounded to fp16. The experts also go to sidx (shared memory), if given.
 template <int PL>
-__device__ __forceinline__ void topk_token(const RouteArgs& a, int t, int lane) {
-  const float* l = a.logits + (size_t)t * a.E;
+__device__ __forceinline__ void topk_token(const RouteArgs& a, const float* l, int t, int lane, int* sidx) {
   float lv[PL];
   unsigned taken = 0;
 #pragma unroll
@@ -157,55 +157,125 @@ __device__ __forceinline__ void topk_token(const RouteArgs& a, int t, int lane) 
     ir[r] = bi;
     zsum += zr[r];
   }
-  if (lane == 0) {
-    for (int r = 0; r < a.k; ++r) {
-      a.idx[t * a.k + r] = ir[r];
-      const float sc = a.scale != nullptr ? a.scale[ir[r]] : 1.0f;
-      a.w[t * a.k + r] = __half2float(__float2half_rn(zr[r] / zsum * sc));
-    }
+  if (lane < a.k) {   // lane r stores rank r
+    float z = 0.f;
+    int e = 0;
+    for (int r = 0; r < a.k; ++r)
+      if (r == lane) { z = zr[r]; e = ir[r]; }
+    const float sc = a.scale != nullptr ? a.scale[e] : 1.0f;
+    a.idx[t * a.k + lane] = e;
+    a.w[t * a.k + lane] = __half2float(__float2half_rn(z / zsum * sc));
+    if (sidx != nullptr) sidx[t * a.k + lane] = e;
   }
 }
 
-// One CTA: a warp per token for the top-k, then the stable expert-grouped
-// order of the pairs p = t*k + r (counts, offsets, union, placement by warp 0).
+// Experts up to which placement runs with a per-warp count table.
+constexpr int kWarpTableE = 128;
+
+// Shared memory of k_route (ints): counts, running, offsets, the per-warp
+// table, the experts of the pairs and, when staged, the logits.
+__host__ __device__ inline size_t route_smem_ints(int M, int E, int k, bool stage_idx, bool stage_logits) {
+  return (size_t)(3 * E + 1) + (E <= kWarpTableE ? 32 * (size_t)E : 0) + (stage_idx ? (size_t)M * k : 0) +
+         (stage_logits ? (size_t)M * E : 0);
+}
+
+// One CTA: a warp per token for the top-k (logits staged in shared memory
+// when they fit), then the stable expert-grouped order of the pairs
+// p = t*k + r: warp-aggregated counts, offsets and union, and the placement,
+// chunk by chunk of the block's threads: a pair's position is its expert's
+// offset, plus the pairs of that expert in earlier chunks, earlier warps of
+// the chunk (a per-warp count table with a prefix over warps) and earlier
+// lanes of its warp (match_any).
 template <int PL>
-__global__ void __launch_bounds__(1024) k_route(const RouteArgs a) {
+__global__ void __launch_bounds__(1024) k_route(const RouteArgs a, int stage_idx, int stage_logits) {
   extern __shared__ int sm[];
   pdl_launch_dependents();
   pdl_wait();
-  int* counts = sm;                 // [E]
-  int* running = sm + a.E;          // [E]
-  int* offs = sm + 2 * a.E;         // [E+1]
-  const int P = a.M * a.k;
+  const int E = a.E, P = a.M * a.k;
+  const bool table = E <= kWarpTableE;
+  int* counts = sm;                                   // [E]
+  int* running = counts + E;                          // [E]
+  int* offs = running + E;                            // [E+1]
+  int* wc = offs + E + 1;                             // [32][E] (table)
+  int* sidx = wc + (table ? 32 * E : 0);              // [P] (stage_idx)
+  float* slog = reinterpret_cast<float*>(sidx + (stage_idx ? P : 0));   // [M][E] (stage_logits)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
 
-  for (int t = warp; t < a.M; t += nwarps) topk_token<PL>(a, t, lane);
-  for (int e = threadIdx.x; e < a.E; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
+  const float* lg = a.logits;
+  if (stage_logits) {
+    for (int i = threadIdx.x; i < a.M * E; i += blockDim.x) slog[i] = a.logits[i];
+    lg = slog;
+  }
+  for (int e = threadIdx.x; e < E; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
+  __syncthreads();
+  for (int t = warp; t < a.M; t += nwarps) topk_token<PL>(a, lg + (size_t)t * E, t, lane, stage_idx ? sidx : nullptr);
   __syncthreads();
   if (a.perm == nullptr) return;
-  for (int p = threadIdx.x; p < P; p += blockDim.x) atomicAdd(&counts[a.idx[p]], 1);
+  const int* pidx = stage_idx ? sidx : a.idx;
+  for (int base = warp * 32; base < P; base += nwarps * 32) {   // warp-aggregated counts
+    const int p = base + lane;
+    const bool act = p < P;
+    const unsigned active = __ballot_sync(0xffffffffu, act);
+    if (act) {
+      const int e = pidx[p];
+      const unsigned same = __match_any_sync(active, e);
+      if ((same & ((1u << lane) - 1u)) == 0) atomicAdd(&counts[e], __popc(same));
+    }
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0, nu = 0;
-    for (int e = 0; e < a.E; ++e) {
+    for (int e = 0; e < E; ++e) {
       offs[e] = acc;
       acc += counts[e];
       if (counts[e] > 0 && a.union_list != nullptr) a.union_list[nu++] = e;
     }
-    offs[a.E] = acc;
+    offs[E] = acc;
     if (a.n_union != nullptr) *a.n_union = nu;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e <= a.E; e += blockDim.x) a.offsets[e] = offs[e];
-  // Stable placement: warp 0 walks the pairs in order, 32 at a time; equal
-  // experts inside a chunk are ranked by lane (match_any + popc).
-  if (threadIdx.x < 32) {
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = offs[e];
+  if (table) {
+    for (int base = 0; base < P; base += blockDim.x) {
+      for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wc[i] = 0;
+      __syncthreads();
+      const int p = base + threadIdx.x;
+      const bool act = p < P;
+      const unsigned active = __ballot_sync(0xffffffffu, act);
+      int e = 0, rank = 0;
+      if (act) {
+        e = pidx[p];
+        const unsigned same = __match_any_sync(active, e);
+        rank = __popc(same & ((1u << lane) - 1u));
+        if (rank == 0) wc[warp * E + e] = __popc(same);
+      }
+      __syncthreads();
+      for (int e2 = threadIdx.x; e2 < E; e2 += blockDim.x) {   // exclusive prefix over warps
+        int s = running[e2];
+        for (int w = 0; w < nwarps; ++w) {
+          const int c = wc[w * E + e2];
+          wc[w * E + e2] = s;
+          s += c;
+        }
+        running[e2] = s;
+      }
+      __syncthreads();
+      if (act) {
+        const int pos = offs[e] + wc[warp * E + e] + rank;
+        a.perm[pos] = p;
+        if (a.inv != nullptr) a.inv[p] = pos;
+      }
+      __syncthreads();
+    }
+  } else if (threadIdx.x < 32) {
+    // Many experts: warp 0 walks the pairs in order, 32 at a time; equal
+    // experts inside a chunk are ranked by lane (match_any + popc).
     for (int base = 0; base < P; base += 32) {
       const int p = base + lane;
       const bool act = p < P;
       const unsigned active = __ballot_sync(0xffffffffu, act);
       if (act) {
-        const int e = a.idx[p];
+        const int e = pidx[p];
         const unsigned same = __match_any_sync(active, e);
         const int rank = __popc(same & ((1u << lane) - 1u));
         const int pos = offs[e] + running[e] + rank;
@@ -246,15 +316,29 @@ cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t s) {
   return launch_pdl(k_router_logits, dim3(a.M, rows), dim3(kRouterThreads), 0, s, a);
 }
 
-cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)(3 * a.E + 1) * sizeof(int);
+namespace {
+template <int PL>
+cudaError_t launch_route_t(const RouteArgs& a, cudaStream_t s) {
+  constexpr size_t kBudget = 200 * 1024;
+  const bool stage_idx = route_smem_ints(a.M, a.E, a.k, true, false) * sizeof(int) <= kBudget;
+  const bool stage_logits = stage_idx && route_smem_ints(a.M, a.E, a.k, true, true) * sizeof(int) <= kBudget;
+  const size_t smem = route_smem_ints(a.M, a.E, a.k, stage_idx, stage_logits) * sizeof(int);
+  if (smem > kBudget) return cudaErrorInvalidValue;   // more experts than the count table and its fallback fit
+  static bool opted[64] = {};
+  const cudaError_t e = opt_in_smem(k_route<PL>, (int)kBudget, opted);
+  if (e != cudaSuccess) return e;
   const int threads = std::min(1024, std::max(128, a.M * 32));   // a warp per token
+  return launch_pdl(k_route<PL>, dim3(1), dim3(threads), smem, s, a, (int)stage_idx, (int)stage_logits);
+}
+}  // namespace
+
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   const int pl = (a.E + 31) / 32;
-  if (pl <= 1) return launch_pdl(k_route<1>, dim3(1), dim3(threads), smem, s, a);
-  if (pl <= 2) return launch_pdl(k_route<2>, dim3(1), dim3(threads), smem, s, a);
-  if (pl <= 4) return launch_pdl(k_route<4>, dim3(1), dim3(threads), smem, s, a);
-  if (pl <= 8) return launch_pdl(k_route<8>, dim3(1), dim3(threads), smem, s, a);
-  return launch_pdl(k_route<32>, dim3(1), dim3(threads), smem, s, a);
+  if (pl <= 1) return launch_route_t<1>(a, s);
+  if (pl <= 2) return launch_route_t<2>(a, s);
+  if (pl <= 4) return launch_route_t<4>(a, s);
+  if (pl <= 8) return launch_route_t<8>(a, s);
+  return launch_route_t<32>(a, s);
 }
 
 }  // namespace moeffn

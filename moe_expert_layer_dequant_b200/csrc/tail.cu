@@ -33,30 +33,56 @@ __device__ __forceinline__ float sum_splits(const float* d, int splits, size_t s
   return h;
 }
 
+// Four consecutive features per thread (16-byte partial loads); N % 4 == 0.
 __global__ void k_tail_elementwise(const TailArgs a) {
   pdl_launch_dependents();
   pdl_wait();
-  const size_t total = (size_t)a.M * a.N;
-  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+  const size_t total4 = (size_t)a.M * a.N / 4;
+  const size_t rstride = (size_t)a.slots * a.N, sstride = (size_t)a.M * a.N;
+  for (size_t i4 = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i4 < total4; i4 += (size_t)gridDim.x * blockDim.x) {
+    const size_t i = 4 * i4;
     const int t = (int)(i / a.N), n = (int)(i - (size_t)t * a.N);
-    float y;
+    float y[4];
     if (a.mode == TAIL_RESIDUAL) {
-      y = round_bf16(sum_splits(a.d, a.splits, (size_t)a.slots * a.N, (size_t)t * a.N + n));
+      float4 h = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < a.splits; ++sp) {   // fixed split order
+        const float4 v = *reinterpret_cast<const float4*>(a.d + sp * rstride + (size_t)t * a.N + n);
+        h.x += v.x; h.y += v.y; h.z += v.z; h.w += v.w;
+      }
+      y[0] = round_bf16(h.x); y[1] = round_bf16(h.y); y[2] = round_bf16(h.z); y[3] = round_bf16(h.w);
     } else {
-      float acc = 0.f;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
       if (a.d_s != nullptr) {
-        const float s = round_bf16(sum_splits(a.d_s, a.splits_s, (size_t)a.M * a.N, (size_t)t * a.N + n));
-        acc = round_bf16(s * sigmoid_f(a.gate_logit[t]));
+        float4 sh = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < a.splits_s; ++sp) {
+          const float4 v = *reinterpret_cast<const float4*>(a.d_s + sp * sstride + (size_t)t * a.N + n);
+          sh.x += v.x; sh.y += v.y; sh.z += v.z; sh.w += v.w;
+        }
+        const float g = sigmoid_f(a.gate_logit[t]);
+        acc[0] = round_bf16(round_bf16(sh.x) * g); acc[1] = round_bf16(round_bf16(sh.y) * g);
+        acc[2] = round_bf16(round_bf16(sh.z) * g); acc[3] = round_bf16(round_bf16(sh.w) * g);
       }
-      for (int r = 0; r < a.k; ++r) {
+      for (int r = 0; r < a.k; ++r) {   // seed first, then the ranks in order
         const int slot = a.inv[t * a.k + r];
-        const float dr = sum_splits(a.d, a.splits, (size_t)a.slots * a.N, (size_t)slot * a.N + n);
-        acc = __fadd_rn(acc, __fmul_rn(a.w[t * a.k + r], dr));
+        const float wr = a.w[t * a.k + r];
+        float4 d = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < a.splits; ++sp) {
+          const float4 v = *reinterpret_cast<const float4*>(a.d + sp * rstride + (size_t)slot * a.N + n);
+          d.x += v.x; d.y += v.y; d.z += v.z; d.w += v.w;
+        }
+        acc[0] = __fadd_rn(acc[0], __fmul_rn(wr, d.x)); acc[1] = __fadd_rn(acc[1], __fmul_rn(wr, d.y));
+        acc[2] = __fadd_rn(acc[2], __fmul_rn(wr, d.z)); acc[3] = __fadd_rn(acc[3], __fmul_rn(wr, d.w));
       }
-      y = round_bf16(acc);
+      for (int j = 0; j < 4; ++j) y[j] = round_bf16(acc[j]);
     }
-    const float x = bf16_bits_to_float(a.res[i]);
-    a.res[i] = float_to_bf16_bits(x + y);
+    const uint2 rv = *reinterpret_cast<const uint2*>(a.res + i);
+    const uint32_t r01 = rv.x, r23 = rv.y;
+    const float x0 = __uint_as_float(r01 << 16), x1 = __uint_as_float(r01 & 0xFFFF0000u);
+    const float x2 = __uint_as_float(r23 << 16), x3 = __uint_as_float(r23 & 0xFFFF0000u);
+    uint2 ov;
+    ov.x = (uint32_t)float_to_bf16_bits(x0 + y[0]) | ((uint32_t)float_to_bf16_bits(x1 + y[1]) << 16);
+    ov.y = (uint32_t)float_to_bf16_bits(x2 + y[2]) | ((uint32_t)float_to_bf16_bits(x3 + y[3]) << 16);
+    *reinterpret_cast<uint2*>(a.res + i) = ov;
   }
 }
 
@@ -134,8 +160,9 @@ cudaError_t launch_tail(const TailArgs& a, cudaStream_t s) {
   if (a.mode == TAIL_RMSNORM) {
     return launch_pdl(k_tail_rmsnorm, dim3(a.M), dim3(512), 16 * sizeof(float), s, a);
   } else {
-    const size_t total = (size_t)a.M * a.N;
-    int blocks = (int)((total + 255) / 256);
+    if (a.N % 4 != 0) return cudaErrorInvalidValue;
+    const size_t total4 = (size_t)a.M * a.N / 4;
+    int blocks = (int)((total4 + 255) / 256);
     if (blocks > 148 * 8) blocks = 148 * 8;
     return launch_pdl(k_tail_elementwise, dim3(blocks), dim3(256), 0, s, a);
   }

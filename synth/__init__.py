@@ -216,13 +216,13 @@ def zero_like_qweight(fmt: str, N: int, K: int) -> QWeight:
 _T_EXPERT_SCALE, _T_SHARED_NORM = 5, 6
 
 
-def with_down_format(li: LayerInputs, down_fmt: str, seed: int) -> LayerInputs:
+def with_down_format(li: LayerInputs, down_fmt: str, seed: int, int8_scale=(0.001, 0.01)) -> LayerInputs:
     """A dense layer whose down projection is stored in another block format
     (per-tensor block types, as in a mixed quantized file)."""
     c = li.config
     out = replace(li)
     out.ffn = FFNWeights(li.ffn.gate, li.ffn.up,
-                         random_qweight(down_fmt, c.H, c.I, _rng(c.cfg, seed, _T_DENSE + 2)))
+                         random_qweight(down_fmt, c.H, c.I, _rng(c.cfg, seed, _T_DENSE + 2), int8_scale=int8_scale))
     return out
 
 

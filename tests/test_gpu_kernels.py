@@ -155,7 +155,8 @@ def test_dense_mixed_block_types(cfg, shape, down_fmt, M):
     """Block types resolved per tensor: the down projection in another format
     than gate and up (GEMV and tensor-core paths)."""
     c = synth.scaled_config(cfg, **shape)
-    inp = synth.with_down_format(synth.make_inputs(c, M, 8), down_fmt, 8)
+    # INT8 down weights scaled like the INT4 ones (|w| ~ 0.1), as a mixed file stores one layer's matrices
+    inp = synth.with_down_format(synth.make_inputs(c, M, 8), down_fmt, 8, int8_scale=(0.0002, 0.002))
     dl = DeviceLayer(inp)
     assert_bf16_close(dl.run(inp.x, inp.residual), oracle.layer(inp), "out")
 
