@@ -239,7 +239,7 @@ struct MoeWS {
   float* d_s;
   uint16_t* xg;      // token rows in pair-slot order (grouped GEMM operand)
   uint16_t* m;       // [M][H] the normed input, when the layer applies its input norm
-  int* cnt;          // [kSMs] arrival counters of phase 2's row ranges (tail folded into phase 2)
+  int* route_cnt;    // [1] arrival counter of the top-k CTAs (zeroed by the router kernel)
 };
 
 // Down-projection K split shared by the routed and the shared expert jobs.
@@ -274,11 +274,12 @@ MoeWS carve_moe(Carve& c, int M, int H, int Ie, int Is, int E, int k) {
   w.d_s = c.take<float>((size_t)sp.shared * M * H);
   w.xg = c.take<uint16_t>(P * H);
   w.m = c.take<uint16_t>((size_t)M * H);
-  w.cnt = c.take<int>(kSMs);
+  w.route_cnt = c.take<int>(1);
   return w;
 }
 
 struct RouterWS {
+  int* counter;      // [1] arrival counter of the top-k CTAs
   float* logits;
   int* perm;
   int* offsets;
@@ -286,6 +287,7 @@ struct RouterWS {
 
 RouterWS carve_router(Carve& c, int M, int E, int k) {
   RouterWS w;
+  w.counter = c.take<int>(1);
   w.logits = c.take<float>((size_t)M * E);
   w.perm = c.take<int>((size_t)M * k);
   w.offsets = c.take<int>(E + 1);
@@ -714,6 +716,7 @@ int moe_router_topk(const moeffn_qweight* router, const uint16_t* x, int M, int 
   ra.H = H;
   ra.E = E;
   ra.logits = logits_out != nullptr ? logits_out : w.logits;
+  ra.route_cnt = w.counter;
   {
     ProfScope ps("router_logits", s);
     MOEFFN_CHECK_CUDA(launch_router_logits(ra, s), "router launch");
@@ -727,6 +730,7 @@ int moe_router_topk(const moeffn_qweight* router, const uint16_t* x, int M, int 
   rt.w = topk_w;
   rt.perm = perm;
   rt.offsets = expert_offsets;
+  rt.counter = w.counter;
   {
     ProfScope ps("route_topk", s);
     MOEFFN_CHECK_CUDA(launch_route(rt, s), "top-k launch");
@@ -921,6 +925,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
   ra.E = E;
   ra.logits = w.logits;
   ra.gate_logit = w.gate_logit;
+  ra.route_cnt = w.route_cnt;
   if (norm_w != nullptr) {   // the router kernel forms m for every later step
     ra.norm_w = norm_w;
     ra.eps = eps;
@@ -945,6 +950,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
   rt.union_list = w.union_list;
   rt.n_union = w.n_union;
   rt.scale = p->expert_scale;
+  rt.counter = w.route_cnt;
   {
     ProfScope ps("route_topk", s);
     MOEFFN_CHECK_CUDA(launch_route(rt, s), "route launch");
@@ -959,7 +965,6 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
   const TmaGeom gu = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, H, max_tok);
   const TmaGeom dn = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 1, sp.ks_len, max_tok);
   int tc_splits_r = splits_r, tc_splits_s = splits_sh;
-  bool tail_done = false;   // the tail ran inside phase 2
   const bool use_tc = p->tc && M >= kTcMinMoeTokens && aligned16(x);
   if (use_tc) {
     // Token rows in pair-slot order feed phase 1's B operand.
@@ -1073,13 +1078,6 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     g.ctas_per_job = std::max(1, kSMs / jobs);
     g.stage_tokens = gu.tokens;
     g.stages = gu.stages;
-    // Qwen form: the seeded rank-ordered tail runs in phase 2's last CTA of
-    // each row range (phase 1 clears the arrival counters).
-    const bool fold_tail = p->shared_post_norm == nullptr;
-    if (fold_tail) {
-      g.zero_cnt = w.cnt;
-      g.zero_n = kSMs;
-    }
     {
       ProfScope ps("phase1_gateup_gemv_tma", s);
       MOEFFN_CHECK_CUDA(launch_tma_gemv(g, 2, gu.mt, 1, jobs, s), "phase-1 launch");
@@ -1113,16 +1111,6 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     d.ctas_per_job = std::max(1, kSMs / (jobs * splits));
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;
-    if (fold_tail) {
-      d.tile_cnt = w.cnt;
-      d.moe_res = residual;
-      d.gate_logit = w.gate_logit;
-      d.route_w = w.w;
-      d.inv = w.inv;
-      d.splits_r = splits_r;
-      d.splits_s = splits_sh;
-      tail_done = true;
-    }
     {
       ProfScope ps("phase2_down_gemv_tma", s);
       MOEFFN_CHECK_CUDA(launch_tma_gemv(d, 1, dn.mt, splits, jobs, s), "phase-2 launch");
@@ -1188,7 +1176,6 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
   }
   }
 
-  if (tail_done) return MOEFFN_OK;
   TailArgs t{};
   t.mode = p->shared_post_norm != nullptr ? TAIL_MOE_GEMMA : TAIL_MOE;
   t.norm_w = p->shared_post_norm;

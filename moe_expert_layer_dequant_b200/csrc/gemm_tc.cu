@@ -17,10 +17,13 @@
 //  warp 0      weight producer: TMA loads of the quantized weight stages (codes
 //              in 128-byte swizzled boxes, INT4 group scales and mins), both
 //              A tiles;
-//  warp 1      allocates TMEM and issues tcgen05.mma (one thread); releases
-//              A and B slots with tcgen05.commit;
+//  warp 1      allocates TMEM; one thread issues tile 0's tcgen05.mma;
 //  warp 2      token producer: TMA loads of the bf16 token tiles (128-byte
 //              swizzled, K = 64 per stage), the MMA's B operand;
+//  warp 3      one thread issues tile 1's tcgen05.mma (the two accumulators
+//              are independent; issuing from two threads halves the per-stage
+//              issue time); A and B slots are released once both issuers'
+//              tcgen05.commit have arrived;
 //  warps 4-19  dequantize, in two sets of eight taking the A stages (K = 64)
 //              in turn: a thread owns one weight row of one A tile and turns
 //              the 64 codes of two quantization groups into bf16 (RNE of the
@@ -238,9 +241,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSW; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], kDqWarps); }
-    for (int i = 0; i < kSB; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 1); }
-    for (int i = 0; i < 8; ++i) { mbar_init(&a_full[i], kDqWarps / 2); mbar_init(&a_empty[i], 1); }
-    mbar_init(acc_full, 1);
+    for (int i = 0; i < kSB; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 2); }
+    for (int i = 0; i < 8; ++i) { mbar_init(&a_full[i], kDqWarps / 2); mbar_init(&a_empty[i], 2); }
+    mbar_init(acc_full, 2);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -295,8 +298,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
       }
       for (int b = max(0, issued - kSB); b < issued; ++b) mbar_wait(&b_full[b % kSB], (b / kSB) & 1);
     }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp == 1 || warp == 3) {
+    // ---------------- MMA issuers: warp 1 for A tile 0, warp 3 for tile 1 ----
+    // The two accumulators are independent, so each tile's MMAs come from its
+    // own thread (on its own SM sub-partition); slots are released when both
+    // threads' commits have arrived.
+    const int tl = warp == 1 ? 0 : 1;
     if (lane == 0 && SA >= 2) {
       const uint32_t idesc = idesc_bf16_f32(kTcRowsA, nmma);
       for (int s = 0; s < nA; ++s) {
@@ -306,11 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
         tc_fence_after();
         const uint64_t bd = umma_desc_sw128(b_base + bs * kBStageBytes);
         const uint32_t acol = tmem + a_col0 + (uint32_t)(slot * kAStageCols);
+        if (tl < tiles) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          for (int t = 0; t < tiles; ++t)
-            umma_bf16_ts(tmem + (uint32_t)(t * ntile), acol + (uint32_t)(t * 32 + kk * 8), bd + 2 * kk, idesc,
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16_ts(tmem + (uint32_t)(tl * ntile), acol + (uint32_t)(tl * 32 + kk * 8), bd + 2 * kk, idesc,
                          (s | kk) != 0);
+        }
         umma_commit(&a_empty[slot]);
         umma_commit(&b_empty[bs]);
       }

@@ -374,46 +374,6 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
       }
     }
   }
-
-  if (a.moe_res != nullptr) {
-    // MoE tail folded in: every routed expert's and the shared expert's K
-    // splits write this row range; the last of them to finish forms, per
-    // token, seed = bf16(bf16(s) * sigmoid(gate logit)) (0 without a shared
-    // expert), adds w_r * d_r for the ranks r = 0..k-1 in order (fp32) and
-    // adds bf16 of the sum to the residual: the arithmetic of the tail kernel.
-    __threadfence();
-    consumer_sync(nthreads);
-    int* last = reinterpret_cast<int*>(xi);   // staged activations are no longer read
-    if (threadIdx.x == 0) {
-      const int expected = *a.n_union * a.splits_r + (a.Ns > 0 ? a.splits_s : 0);
-      const int old = atomicAdd(&a.tile_cnt[blockIdx.x], 1);
-      *last = old == expected - 1;
-      if (*last) a.tile_cnt[blockIdx.x] = 0;  // ready for the next call
-    }
-    consumer_sync(nthreads);
-    if (*last) {
-      __threadfence();
-      const int nr = r1 - r0, N = job.N;
-      const size_t rstride = (size_t)a.slots * N, sstride = (size_t)a.M * N;
-      for (int i = threadIdx.x; i < nr * a.M; i += nthreads) {
-        const int t = i / nr, n = r0 + (i - t * nr);
-        float acc = 0.f;
-        if (a.Ns > 0) {   // a shared expert seeds the sum
-          float sh = 0.f;
-          for (int sp = 0; sp < a.splits_s; ++sp) sh += __ldcg(a.out_d_s + sp * sstride + (size_t)t * N + n);
-          acc = round_bf16(round_bf16(sh) * sigmoid_f(__ldcg(a.gate_logit + t)));
-        }
-        for (int r = 0; r < a.topk; ++r) {
-          const int slot = __ldcg(a.inv + t * a.topk + r);
-          float dr = 0.f;
-          for (int sp = 0; sp < a.splits_r; ++sp) dr += __ldcg(a.out_d + sp * rstride + (size_t)slot * N + n);
-          acc = __fadd_rn(acc, __fmul_rn(__ldcg(a.route_w + t * a.topk + r), dr));
-        }
-        const size_t o = (size_t)t * N + n;
-        a.moe_res[o] = float_to_bf16_bits(bf16_bits_to_float(a.moe_res[o]) + round_bf16(acc));
-      }
-    }
-  }
 }
 
 template <int FMT, int MT, int NM>

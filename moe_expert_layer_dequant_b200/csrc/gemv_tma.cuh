@@ -57,15 +57,6 @@ struct TmaGemvArgs {
   int* tile_cnt;               // down, dense mode: arrivals of the K splits per CTA row range
   uint16_t* res;               // down, dense mode: residual [M][N], updated in place by the last K split
                                // of each row range (null: fp32 partials only, a tail kernel adds them)
-  // Down, grouped mode (MoE phase 2, Qwen form): the last CTA to finish a row
-  // range, over every routed expert's and the shared expert's jobs and K
-  // splits, adds the seeded rank-ordered sum of that range to moe_res in place
-  // (null: a tail kernel does it). Arrivals are counted in tile_cnt.
-  uint16_t* moe_res;           // [M][N]
-  const float* gate_logit;     // [M] shared-expert gate logits (with a shared expert)
-  const float* route_w;        // [M][k] routing weights
-  const int* inv;              // [M*k] slot of pair p
-  int splits_r, splits_s;      // K splits of the routed and the shared jobs
   const uint16_t* norm_w;      // dense gate/up, unsplit K: normalize x on staging (RMSNorm weight [K]), or null
   float eps;
   int ks_len;                  // K elements per split (INT4: multiple of 256)

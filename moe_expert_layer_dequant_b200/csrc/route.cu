@@ -29,6 +29,7 @@ __global__ void __launch_bounds__(kRouterThreads) k_router_logits(const RouterAr
   pdl_wait();
   const int t = blockIdx.x;
   const int e = blockIdx.y;
+  if (a.route_cnt != nullptr && t == 0 && e == 0 && threadIdx.x == 0) *a.route_cnt = 0;   // for the top-k kernel next
   const bool gate_row = (e == a.E);
   const uint16_t* x = a.x + (size_t)t * a.H;
   const bool norm = a.norm_w != nullptr;
@@ -171,53 +172,37 @@ __device__ __forceinline__ void topk_token(const RouteArgs& a, const float* l, i
 
 // Experts up to which placement runs with a per-warp count table.
 constexpr int kWarpTableE = 128;
+constexpr int kRouteWarps = 8;   // tokens (warps) per top-k CTA
 
-// Shared memory of k_route (ints): counts, running, offsets, the per-warp
-// table, the experts of the pairs and, when staged, the logits.
-__host__ __device__ inline size_t route_smem_ints(int M, int E, int k, bool stage_idx, bool stage_logits) {
-  return (size_t)(3 * E + 1) + (E <= kWarpTableE ? 32 * (size_t)E : 0) + (stage_idx ? (size_t)M * k : 0) +
-         (stage_logits ? (size_t)M * E : 0);
+// Shared memory of the placing CTA (ints): counts, running, offsets and the
+// per-warp count table.
+__host__ __device__ inline size_t route_smem_ints(int E) {
+  return (size_t)(3 * E + 1) + (E <= kWarpTableE ? (size_t)kRouteWarps * E : 0);
 }
 
-// One CTA: a warp per token for the top-k (logits staged in shared memory
-// when they fit), then the stable expert-grouped order of the pairs
-// p = t*k + r: warp-aggregated counts, offsets and union, and the placement,
-// chunk by chunk of the block's threads: a pair's position is its expert's
-// offset, plus the pairs of that expert in earlier chunks, earlier warps of
-// the chunk (a per-warp count table with a prefix over warps) and earlier
-// lanes of its warp (match_any).
-template <int PL>
-__global__ void __launch_bounds__(1024) k_route(const RouteArgs a, int stage_idx, int stage_logits) {
-  extern __shared__ int sm[];
-  pdl_launch_dependents();
-  pdl_wait();
+// The stable expert-grouped order of the pairs p = t*k + r, by one CTA:
+// warp-aggregated counts, offsets and union, then the placement chunk by
+// chunk of the block's threads -- a pair's position is its expert's offset,
+// plus the pairs of that expert in earlier chunks, in earlier warps of the
+// chunk (a per-warp count table with a prefix over warps) and in earlier
+// lanes of its warp (match_any). Experts come from global memory (written by
+// other CTAs: read through L2).
+__device__ void place_pairs(const RouteArgs& a, int* sm) {
   const int E = a.E, P = a.M * a.k;
   const bool table = E <= kWarpTableE;
   int* counts = sm;                                   // [E]
   int* running = counts + E;                          // [E]
   int* offs = running + E;                            // [E+1]
-  int* wc = offs + E + 1;                             // [32][E] (table)
-  int* sidx = wc + (table ? 32 * E : 0);              // [P] (stage_idx)
-  float* slog = reinterpret_cast<float*>(sidx + (stage_idx ? P : 0));   // [M][E] (stage_logits)
+  int* wc = offs + E + 1;                             // [kRouteWarps][E] (table)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
-
-  const float* lg = a.logits;
-  if (stage_logits) {
-    for (int i = threadIdx.x; i < a.M * E; i += blockDim.x) slog[i] = a.logits[i];
-    lg = slog;
-  }
   for (int e = threadIdx.x; e < E; e += blockDim.x) { counts[e] = 0; running[e] = 0; }
   __syncthreads();
-  for (int t = warp; t < a.M; t += nwarps) topk_token<PL>(a, lg + (size_t)t * E, t, lane, stage_idx ? sidx : nullptr);
-  __syncthreads();
-  if (a.perm == nullptr) return;
-  const int* pidx = stage_idx ? sidx : a.idx;
   for (int base = warp * 32; base < P; base += nwarps * 32) {   // warp-aggregated counts
     const int p = base + lane;
     const bool act = p < P;
     const unsigned active = __ballot_sync(0xffffffffu, act);
     if (act) {
-      const int e = pidx[p];
+      const int e = __ldcg(a.idx + p);
       const unsigned same = __match_any_sync(active, e);
       if ((same & ((1u << lane) - 1u)) == 0) atomicAdd(&counts[e], __popc(same));
     }
@@ -237,14 +222,14 @@ __global__ void __launch_bounds__(1024) k_route(const RouteArgs a, int stage_idx
   for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = offs[e];
   if (table) {
     for (int base = 0; base < P; base += blockDim.x) {
-      for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) wc[i] = 0;
+      for (int i = threadIdx.x; i < nwarps * E; i += blockDim.x) wc[i] = 0;
       __syncthreads();
       const int p = base + threadIdx.x;
       const bool act = p < P;
       const unsigned active = __ballot_sync(0xffffffffu, act);
       int e = 0, rank = 0;
       if (act) {
-        e = pidx[p];
+        e = __ldcg(a.idx + p);
         const unsigned same = __match_any_sync(active, e);
         rank = __popc(same & ((1u << lane) - 1u));
         if (rank == 0) wc[warp * E + e] = __popc(same);
@@ -275,7 +260,7 @@ __global__ void __launch_bounds__(1024) k_route(const RouteArgs a, int stage_idx
       const bool act = p < P;
       const unsigned active = __ballot_sync(0xffffffffu, act);
       if (act) {
-        const int e = pidx[p];
+        const int e = __ldcg(a.idx + p);
         const unsigned same = __match_any_sync(active, e);
         const int rank = __popc(same & ((1u << lane) - 1u));
         const int pos = offs[e] + running[e] + rank;
@@ -287,6 +272,32 @@ __global__ void __launch_bounds__(1024) k_route(const RouteArgs a, int stage_idx
       __syncwarp();
     }
   }
+}
+
+// Top-k of kRouteWarps tokens per CTA (a warp each); the last CTA to finish
+// (an arrival counter, zeroed by the kernel that runs before: the router, or
+// the caller) places the pairs of all tokens.
+template <int PL>
+__global__ void __launch_bounds__(32 * kRouteWarps) k_route(const RouteArgs a) {
+  extern __shared__ int sm[];
+  __shared__ int s_last;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kRouteWarps + warp;
+  if (t < a.M) topk_token<PL>(a, a.logits + (size_t)t * a.E, t, lane, nullptr);
+  if (a.perm == nullptr) return;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int old = atomicAdd(a.counter, 1);
+    s_last = old == (int)gridDim.x - 1;
+    if (s_last) *a.counter = 0;   // ready for the next call
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  place_pairs(a, sm);
 }
 
 // Token rows in expert-grouped pair order: the B operand rows of the grouped
@@ -319,16 +330,10 @@ cudaError_t launch_router_logits(const RouterArgs& a, cudaStream_t s) {
 namespace {
 template <int PL>
 cudaError_t launch_route_t(const RouteArgs& a, cudaStream_t s) {
-  constexpr size_t kBudget = 200 * 1024;
-  const bool stage_idx = route_smem_ints(a.M, a.E, a.k, true, false) * sizeof(int) <= kBudget;
-  const bool stage_logits = stage_idx && route_smem_ints(a.M, a.E, a.k, true, true) * sizeof(int) <= kBudget;
-  const size_t smem = route_smem_ints(a.M, a.E, a.k, stage_idx, stage_logits) * sizeof(int);
-  if (smem > kBudget) return cudaErrorInvalidValue;   // more experts than the count table and its fallback fit
-  static bool opted[64] = {};
-  const cudaError_t e = opt_in_smem(k_route<PL>, (int)kBudget, opted);
-  if (e != cudaSuccess) return e;
-  const int threads = std::min(1024, std::max(128, a.M * 32));   // a warp per token
-  return launch_pdl(k_route<PL>, dim3(1), dim3(threads), smem, s, a, (int)stage_idx, (int)stage_logits);
+  const size_t smem = route_smem_ints(a.E) * sizeof(int);
+  if (a.perm != nullptr && a.counter == nullptr) return cudaErrorInvalidValue;
+  const int blocks = (a.M + kRouteWarps - 1) / kRouteWarps;
+  return launch_pdl(k_route<PL>, dim3(blocks), dim3(32 * kRouteWarps), smem, s, a);
 }
 }  // namespace
 

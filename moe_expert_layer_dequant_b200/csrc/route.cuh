@@ -20,6 +20,7 @@ struct RouterArgs {
   const uint16_t* norm_w;
   float eps;
   uint16_t* m_out;
+  int* route_cnt;              // zeroed here for the top-k kernel that follows, or null
 };
 
 // m = rms_norm(x, w) row by row into m [M][H] (one CTA per row).
@@ -43,6 +44,7 @@ struct RouteArgs {
   int* union_list;             // [E] or null
   int* n_union;                // [1] or null
   const float* scale;          // [E] per-expert scale of the routing weights, or null (ones)
+  int* counter;                // [1] arrival counter of the top-k CTAs, zero on entry (with perm)
 };
 
 // xg[s][:] = x[perm[s] / topk][:] for the P = M*topk pair slots (bf16 rows of H).

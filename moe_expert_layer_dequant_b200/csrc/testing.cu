@@ -15,6 +15,8 @@ int api_fail(int code, const char* msg);
 
 namespace {
 
+__device__ int g_test_route_counter = 0;   // arrival counter of the test export's top-k CTAs
+
 // One thread per 32-bit word of codes: 8 INT4 codes or 4 INT8 codes.
 __global__ void k_dequant(const QW w, int fmt, int N, int K, float* out_f32, uint16_t* out_bf16) {
   const int per_word = fmt == FMT_INT4_G32 ? 8 : 4;
@@ -78,7 +80,16 @@ int moeffn_test_topk_from_logits(const float* logits, int M, int E, int top_k, i
   a.offsets = expert_offsets;
   a.union_list = union_out;
   a.n_union = n_union_out;
-  const cudaError_t e = launch_route(a, reinterpret_cast<cudaStream_t>(stream));
+  // The top-k CTAs count their arrivals in a counter that must start at zero.
+  static int* counter[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return api_fail(MOEFFN_ERR_CUDA, "test_topk: device");
+  if (counter[dev] == nullptr && cudaGetSymbolAddress(reinterpret_cast<void**>(&counter[dev]), g_test_route_counter) != cudaSuccess)
+    return api_fail(MOEFFN_ERR_CUDA, "test_topk: counter address");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(counter[dev], 0, sizeof(int), st) != cudaSuccess) return api_fail(MOEFFN_ERR_CUDA, "test_topk: memset");
+  a.counter = counter[dev];
+  const cudaError_t e = launch_route(a, st);
   if (e != cudaSuccess) return api_fail(MOEFFN_ERR_CUDA, cudaGetErrorString(e));
   return MOEFFN_OK;
 }
