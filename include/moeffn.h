@@ -44,6 +44,16 @@
  *  - MOEFFN_Q_INT4_AFFINE_G32: q = uint8 [rows][cols/2], element 2j in the low
  *    nibble of byte j, 2j+1 in the high nibble; scale, min = fp16
  *    [rows][cols/32]. W[n][k] = q * scale[n][k/32] + min[n][k/32]. cols % 32 == 0.
+ *  - MOEFFN_Q_Q4_K: the K-quant block type of Q4_K_M files (turbospark-runtime
+ *    0.3.0, src/families/llama/dense.rs: encode_gemv_any resolves the block
+ *    type of each tensor), in the public GGUF layout, which the pages do not
+ *    spell out. q = [rows][cols/256] super-blocks of 144 bytes: fp16 d (bytes
+ *    0-1), fp16 dmin (2-3), the 6-bit scale and min of the eight 32-weight
+ *    sub-blocks packed in bytes 4-15, then 128 code bytes in four runs of 32
+ *    (run c: weights 64c..64c+31 in the low nibbles, 64c+32..64c+63 in the
+ *    high nibbles). W = fp32(d * scale_j * q - dmin * min_j). scale = min =
+ *    NULL. cols % 256 == 0. Dense layers only (ffn_dense, ffn_shared_expert),
+ *    each of gate/up and down independently.
  *  - MOEFFN_BF16 / MOEFFN_F32: plain [rows][cols] in q (router, gate vector).
  *  All base pointers 16-byte aligned.
  */
@@ -72,7 +82,8 @@ typedef enum {
   MOEFFN_Q_INT8_ROW = 1,
   MOEFFN_Q_INT4_AFFINE_G32 = 2,
   MOEFFN_BF16 = 3,
-  MOEFFN_F32 = 4
+  MOEFFN_F32 = 4,
+  MOEFFN_Q_Q4_K = 5
 } moeffn_qformat;
 
 typedef enum { MOEFFN_ACT_SILU = 0, MOEFFN_ACT_GELU_TANH = 1 } moeffn_act;

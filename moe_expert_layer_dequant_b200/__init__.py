@@ -28,11 +28,11 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoeffn.so")
 
 # moeffn_qformat / moeffn_act / moeffn_kind
-Q_INT8_ROW, Q_INT4_AFFINE_G32, BF16, F32 = 1, 2, 3, 4
+Q_INT8_ROW, Q_INT4_AFFINE_G32, BF16, F32, Q_Q4_K = 1, 2, 3, 4, 5
 ACT_SILU, ACT_GELU_TANH = 0, 1
 KIND_DENSE, KIND_SHARED, KIND_ROUTER, KIND_MOE = 1, 2, 3, 4
 ACTS = {"silu": ACT_SILU, "gelu_tanh": ACT_GELU_TANH}
-FORMATS = {"int8_row": Q_INT8_ROW, "int4_g32": Q_INT4_AFFINE_G32}
+FORMATS = {"int8_row": Q_INT8_ROW, "int4_g32": Q_INT4_AFFINE_G32, "q4_k": Q_Q4_K}
 
 
 class MoeffnError(RuntimeError):

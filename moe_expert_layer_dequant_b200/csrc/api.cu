@@ -65,10 +65,16 @@ QW to_qw(const moeffn_qweight& w) {
 }
 
 int check_qweight(const moeffn_qweight& w, const char* name, int rows, int cols) {
-  if (w.format != MOEFFN_Q_INT8_ROW && w.format != MOEFFN_Q_INT4_AFFINE_G32)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: format %d is not INT8_ROW or INT4_AFFINE_G32", name, w.format);
+  if (w.format != MOEFFN_Q_INT8_ROW && w.format != MOEFFN_Q_INT4_AFFINE_G32 && w.format != MOEFFN_Q_Q4_K)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: format %d is not INT8_ROW, INT4_AFFINE_G32 or Q4_K", name, w.format);
   if (w.rows != rows || w.cols != cols)
     return fail(MOEFFN_ERR_INVALID, "%s: shape [%d][%d], expected [%d][%d]", name, w.rows, w.cols, rows, cols);
+  if (w.format == MOEFFN_Q_Q4_K) {   // scales and mins live in the blocks
+    if (w.q == nullptr) return fail(MOEFFN_ERR_INVALID, "%s: null q", name);
+    if (!aligned16(w.q)) return fail(MOEFFN_ERR_INVALID, "%s: q is not 16-byte aligned", name);
+    if (cols % 256 != 0) return fail(MOEFFN_ERR_INVALID, "%s: Q4_K needs cols %% 256 == 0 (cols=%d)", name, cols);
+    return MOEFFN_OK;
+  }
   if (w.q == nullptr || w.scale == nullptr)
     return fail(MOEFFN_ERR_INVALID, "%s: null q or scale", name);
   if (!aligned16(w.q)) return fail(MOEFFN_ERR_INVALID, "%s: q is not 16-byte aligned", name);
@@ -106,11 +112,12 @@ int rows_per_cta(int rows_total) {
   return std::min(64, std::max(8, r));
 }
 
-// K split of a down projection: slices of at most 4096 (INT4) or 2048 (INT8)
-// elements, a multiple of 256 (16-byte aligned scale rows and TMA boxes of at
-// most 256 eight-byte elements); every split starts below K.
+// K split of a down projection: slices of at most 4096 (INT4), 3584 (Q4_K:
+// 14 blocks of 18 eight-byte elements) or 2048 (INT8) elements, a multiple of
+// 256 (16-byte aligned scale rows and TMA boxes of at most 256 eight-byte
+// elements); every split starts below K.
 int down_slice(int K, int fmt) {
-  const int lim = fmt == MOEFFN_Q_INT8_ROW ? 2048 : 4096;
+  const int lim = fmt == MOEFFN_Q_INT8_ROW ? 2048 : fmt == MOEFFN_Q_Q4_K ? 3584 : 4096;
   const int s = (K + lim - 1) / lim;
   return ((K + s - 1) / s + 255) / 256 * 256;
 }
@@ -120,7 +127,8 @@ int down_splits(int K, int fmt) {
 }
 // Partial-sum buffers are sized for the format with more splits.
 int down_splits_any(int K) {
-  return std::max(down_splits(K, MOEFFN_Q_INT8_ROW), down_splits(K, MOEFFN_Q_INT4_AFFINE_G32));
+  return std::max(std::max(down_splits(K, MOEFFN_Q_INT8_ROW), down_splits(K, MOEFFN_Q_INT4_AFFINE_G32)),
+                  down_splits(K, MOEFFN_Q_Q4_K));
 }
 
 // ---- TMA-fed GEMV eligibility and geometry ---------------------------------
@@ -134,7 +142,7 @@ constexpr size_t kTmaXBudget = 72 * 1024;
 // 0; a matrix split along K loads its scale and min boxes through 2-D tensor
 // maps, whose row stride (K / 16 bytes) must be a multiple of 16: K % 256 == 0.
 bool tma_ok(const moeffn_qweight& w) {
-  if (w.format == MOEFFN_Q_INT8_ROW) return true;
+  if (w.format == MOEFFN_Q_INT8_ROW || w.format == MOEFFN_Q_Q4_K) return true;
   if (w.rows % 8 != 0 || !aligned16(w.scale) || !aligned16(w.min)) return false;
   return w.cols % 256 == 0 || down_splits(w.cols, MOEFFN_Q_INT4_AFFINE_G32) == 1;
 }
@@ -180,6 +188,7 @@ constexpr int kTcMinMoeTokens = 8;   // MoE layer: token rows from which the gro
 bool tc_ok(const moeffn_qweight& w) {
   if (!aligned16(w.q)) return false;
   if (w.format == MOEFFN_Q_INT4_AFFINE_G32) return w.cols % 256 == 0 && aligned16(w.scale) && aligned16(w.min);
+  if (w.format == MOEFFN_Q_Q4_K) return w.cols % 256 == 0;
   return w.format == MOEFFN_Q_INT8_ROW && w.cols % 128 == 0 && aligned16(w.scale);
 }
 bool tc_ok(const moeffn_ffn& f) { return tc_ok(f.gate) && tc_ok(f.up) && tc_ok(f.down); }
@@ -453,6 +462,9 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     return MOEFFN_OK;
   }
 
+  // The register-load GEMV below takes the INT8 and INT4 block types only.
+  if (fmt == MOEFFN_Q_Q4_K || dfmt == MOEFFN_Q_Q4_K)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "Q4_K weights need the bulk-copy GEMV (shape or alignment not eligible)");
   if (norm_w != nullptr) {
     if ((rc = launch_prenorm(x, norm_w, eps, M, H, w, s)) != MOEFFN_OK) return rc;
     x = w.m;

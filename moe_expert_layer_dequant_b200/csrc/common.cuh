@@ -9,13 +9,15 @@
 namespace moeffn {
 
 // Weight formats (values match moeffn_qformat in include/moeffn.h).
-enum : int { FMT_INT8_ROW = 1, FMT_INT4_G32 = 2, FMT_BF16 = 3, FMT_F32 = 4 };
+enum : int { FMT_INT8_ROW = 1, FMT_INT4_G32 = 2, FMT_BF16 = 3, FMT_F32 = 4, FMT_Q4K = 5 };
 enum : int { ACT_SILU = 0, ACT_GELU_TANH = 1 };
 
 // Device view of one quantized matrix W[N][K] (row-major, K contiguous).
 //  INT8-row : q = int8 [N][K], scale = fp16 [N], mn = null.
 //  INT4-g32 : q = uint8 [N][K/2] (element 2j = low nibble of byte j),
 //             scale = fp16 [N][K/32], mn = fp16 [N][K/32]; w = q*scale + mn.
+//  Q4_K     : q = [N][K/256] super-blocks of 144 bytes, scale = mn = null
+//             (see Q4K below).
 struct QW {
   const uint8_t* q;
   const __half* scale;
@@ -149,6 +151,39 @@ __device__ __forceinline__ void int8_word_dequant(uint32_t w, float s, float (&o
     out[i] = q * s;
   }
 }
+
+// Q4_K super-block (the GGUF K-quant layout): 256 weights in 144 bytes,
+//  bytes 0-1 d (fp16), 2-3 dmin (fp16), 4-15 the packed 6-bit scale and min
+//  of sub-blocks 0..7 (32 weights each), 16-143 codes in four runs of 32
+//  bytes: run c holds weights 64c..64c+31 in its low nibbles and
+//  64c+32..64c+63 in its high nibbles. w = d * scale_j * q - dmin * min_j;
+//  d * scale_j and dmin * min_j are exact in fp32, so fmaf(q, d * scale_j,
+//  -dmin * min_j) is the exact value rounded once.
+struct Q4K {
+  static constexpr int kBlock = 256;
+  static constexpr int kBytes = 144;
+  // hdr: the block's first 16 bytes as four words (d | dmin << 16, then the
+  // 12 packed bytes s[0..11]). Sub-blocks 0..3: scale = s[j] & 63, min =
+  // s[j + 4] & 63; 4..7: low 4 bits from the nibbles of s[j + 4], top 2 bits
+  // from the top of s[j - 4] (scale) and s[j] (min).
+  static __device__ __forceinline__ void scale_min(const uint4& hdr, int j, float& sc, float& mn) {
+    const uint32_t lo = hdr.y, mid = hdr.z, hi = hdr.w;   // s[0..3], s[4..7], s[8..11]
+    uint32_t a, b;
+    if (j < 4) {
+      a = (lo >> (8 * j)) & 63u;
+      b = (mid >> (8 * j)) & 63u;
+    } else {
+      const int i = j - 4;
+      const uint32_t h = (hi >> (8 * i)) & 0xFFu;
+      a = (h & 15u) | (((lo >> (8 * i + 6)) & 3u) << 4);
+      b = (h >> 4) | (((mid >> (8 * i + 6)) & 3u) << 4);
+    }
+    const float d = __half2float(__ushort_as_half((unsigned short)(hdr.x & 0xFFFFu)));
+    const float dmin = __half2float(__ushort_as_half((unsigned short)(hdr.x >> 16)));
+    sc = d * (float)a;
+    mn = -(dmin * (float)b);
+  }
+};
 
 }  // namespace moeffn
 

@@ -78,6 +78,16 @@ struct TcFmt<FMT_INT8_ROW> {
   static constexpr int kStageBytes = kTilesA * kTileBytes;
 };
 
+template <>
+struct TcFmt<FMT_Q4K> {
+  static constexpr int kKTile = Q4K::kBlock;                // one super-block per row and stage
+  static constexpr int kGroups = kKTile / 32;
+  static constexpr int kCodeBytes = kTcRowsA * Q4K::kBytes; // unswizzled rows of 144 bytes
+  static constexpr int kScaleBytes = 0;
+  static constexpr int kTileBytes = kCodeBytes;
+  static constexpr int kStageBytes = kTilesA * kTileBytes;
+};
+
 template <int FMT>
 constexpr size_t tc_smem_bytes() {
   return 1024 /*align slack*/ + 1024 /*barriers*/ + (size_t)kSW * TcFmt<FMT>::kStageBytes +
@@ -85,7 +95,9 @@ constexpr size_t tc_smem_bytes() {
 }
 static_assert(tc_smem_bytes<FMT_INT4_G32>() <= 232448, "shared memory");
 static_assert(tc_smem_bytes<FMT_INT8_ROW>() <= 232448, "shared memory");
+static_assert(tc_smem_bytes<FMT_Q4K>() <= 232448, "shared memory");
 static_assert(TcFmt<FMT_INT4_G32>::kStageBytes % 1024 == 0 && TcFmt<FMT_INT8_ROW>::kStageBytes % 1024 == 0 &&
+                  TcFmt<FMT_Q4K>::kStageBytes % 1024 == 0 &&
                   kBStageBytes % 1024 == 0,
               "stage bases stay 1024-byte aligned (128-byte swizzle)");
 
@@ -164,6 +176,43 @@ __device__ __forceinline__ void dq_group_int4(uint32_t tile, int r, int g, uint3
     o[4 * q + 1] = pack_bf16x2(c23.x, c23.y);
     o[4 * q + 2] = pack_bf16x2(c45.x, c45.y);
     o[4 * q + 3] = pack_bf16x2(c67.x, c67.y);
+  }
+}
+
+// Q4_K: A stage a (0..3) of a weight stage is code run a of the row's block:
+// 32 bytes whose low nibbles are the stage's K elements 0..31 (sub-block 2a,
+// into o0) and whose high nibbles are elements 32..63 (sub-block 2a + 1, into
+// o1). Each value is fmaf(q, d * scale, -dmin * min), the exact weight rounded
+// once to fp32, then rounded to bf16. The masks pick the nibbles of bytes 0
+// and 1 (lo) or of their high halves (hi) in place, so the scale is divided by
+// the nibble's place value (exact: a power of two).
+__device__ __forceinline__ void dq_run_q4k(uint32_t tile, int r, int a, uint32_t (&o0)[16], uint32_t (&o1)[16]) {
+  const uint32_t row = tile + r * Q4K::kBytes;
+  const uint4 hdr = lds_u128(row);
+  const uint4 ca = lds_u128(row + 16 + 32 * a), cb = lds_u128(row + 32 + 32 * a);
+  float sl, ml, sh, mh;
+  Q4K::scale_min(hdr, 2 * a, sl, ml);
+  Q4K::scale_min(hdr, 2 * a + 1, sh, mh);
+  const uint32_t mg = kMagic;
+  const float2 sub = make_float2(-kMagicF, -kMagicF);
+  const float2 lo_s = make_float2(sl, sl * 0.00390625f), lo_m = make_float2(ml, ml);
+  const float2 hi_s = make_float2(sh * 0.0625f, sh * 0.000244140625f), hi_m = make_float2(mh, mh);
+  const uint32_t words[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {   // word q: elements 4q..4q+3 of both sub-blocks
+    const uint32_t w = words[q], h = w >> 16;
+    float2 l01 = make_float2(__uint_as_float(and_or(w, 0x000Fu, mg)), __uint_as_float(and_or(w, 0x0F00u, mg)));
+    float2 l23 = make_float2(__uint_as_float(and_or(h, 0x000Fu, mg)), __uint_as_float(and_or(h, 0x0F00u, mg)));
+    float2 h01 = make_float2(__uint_as_float(and_or(w, 0x00F0u, mg)), __uint_as_float(and_or(w, 0xF000u, mg)));
+    float2 h23 = make_float2(__uint_as_float(and_or(h, 0x00F0u, mg)), __uint_as_float(and_or(h, 0xF000u, mg)));
+    l01 = __ffma2_rn(__fadd2_rn(l01, sub), lo_s, lo_m);
+    l23 = __ffma2_rn(__fadd2_rn(l23, sub), lo_s, lo_m);
+    h01 = __ffma2_rn(__fadd2_rn(h01, sub), hi_s, hi_m);
+    h23 = __ffma2_rn(__fadd2_rn(h23, sub), hi_s, hi_m);
+    o0[2 * q] = pack_bf16x2(l01.x, l01.y);
+    o0[2 * q + 1] = pack_bf16x2(l23.x, l23.y);
+    o1[2 * q] = pack_bf16x2(h01.x, h01.y);
+    o1[2 * q + 1] = pack_bf16x2(h23.x, h23.y);
   }
 }
 
@@ -269,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
         uint8_t* gst = gbase + (w_base - base) + slot * F::kStageBytes;
         mbar_arrive_expect_tx(&w_full[slot], tx);
         const int kc = k0 + w * F::kKTile;                  // first K element of the stage
-        const int cx = (FMT == FMT_INT4_G32) ? kc / 2 : kc;  // byte column of the codes
+        const int cx = (FMT == FMT_INT4_G32) ? kc / 2 : (FMT == FMT_Q4K) ? kc / Q4K::kBlock * Q4K::kBytes : kc;  // byte column
         for (int t = 0; t < tiles; ++t) {
           const TcMaps* mp = t == 0 ? job.m0 : job.m1;
           const int rw = t == 0 ? row0 : row1;
@@ -344,6 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
         uint32_t o0[16], o1[16];
         const uint32_t tile = w_base + ws * F::kStageBytes + t * F::kTileBytes;
         if (FMT == FMT_INT4_G32) { dq_group_int4(tile, r, g, o0); dq_group_int4(tile, r, g + 1, o1); }
+        else if (FMT == FMT_Q4K) dq_run_q4k(tile, r, g / 2, o0, o1);
         else { dq_group_int8(tile, r, g, o0); dq_group_int8(tile, r, g + 1, o1); }
         const uint32_t ta = tmem + lane_base + a_col0 + (uint32_t)(slot * kAStageCols + t * 32);
         tmem_st16(ta, o0);
@@ -441,6 +491,13 @@ cudaError_t encode_tc_weight_maps(TcMaps* m, int fmt, const QW& w, int N, int K)
     if (e != cudaSuccess) return e;
     return encode_tmap_2d(&m->mn, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.mn, K / 32, N, K / 16, 8, kTcRowsA);
   }
+  if (fmt == FMT_Q4K) {   // one 144-byte block per row and stage, unswizzled
+    const uint64_t rb = (uint64_t)K / Q4K::kBlock * Q4K::kBytes;
+    e = encode_tmap_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.q, rb, N, rb, Q4K::kBytes, kTcRowsA);
+    m->scale = m->codes;
+    m->mn = m->codes;
+    return e;
+  }
   e = encode_tmap_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, w.q, K, N, K, 128, kTcRowsA,
                      CU_TENSOR_MAP_SWIZZLE_128B);
   m->scale = m->codes;
@@ -459,6 +516,8 @@ cudaError_t launch_tc_gemm(const TcGemmArgs& a, int row_tiles, int splits, int j
   const dim3 grid(row_tiles, a.token_tiles * splits, jobs);
   if (a.fmt == FMT_INT4_G32)
     return a.mode == TC_GATEUP ? launch_t<FMT_INT4_G32, TC_GATEUP>(a, grid, s) : launch_t<FMT_INT4_G32, TC_DOWN>(a, grid, s);
+  if (a.fmt == FMT_Q4K)
+    return a.mode == TC_GATEUP ? launch_t<FMT_Q4K, TC_GATEUP>(a, grid, s) : launch_t<FMT_Q4K, TC_DOWN>(a, grid, s);
   return a.mode == TC_GATEUP ? launch_t<FMT_INT8_ROW, TC_GATEUP>(a, grid, s) : launch_t<FMT_INT8_ROW, TC_DOWN>(a, grid, s);
 }
 

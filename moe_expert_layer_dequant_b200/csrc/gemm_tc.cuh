@@ -13,8 +13,8 @@ constexpr int kTcRowsA = 128;
 constexpr int kTcMaxTok = 192;
 
 // Tensor maps of one quantized matrix for the GEMM, boxes of kTcRowsA rows:
-// codes (uint8, 128-byte swizzled [128 rows][128 bytes]), INT4 scales and
-// mins (u16 [128 rows][8 groups]).
+// codes (uint8, 128-byte swizzled [128 rows][128 bytes]; Q4_K: unswizzled
+// [128 rows][one 144-byte block]), INT4 scales and mins (u16 [128 rows][8 groups]).
 struct TcMaps {
   CUtensorMap codes, scale, mn;
 };
@@ -45,8 +45,8 @@ struct TcGemmArgs {
   int token_tiles;             // grid.y = token_tiles * splits
 };
 
-// K covered by one weight stage: 256 codes (INT4) or 128 (INT8).
-inline int tc_k_tile(int fmt) { return fmt == FMT_INT4_G32 ? 256 : 128; }
+// K covered by one weight stage: 256 codes (INT4, Q4_K) or 128 (INT8).
+inline int tc_k_tile(int fmt) { return fmt == FMT_INT8_ROW ? 128 : 256; }
 // Output features per CTA (GATEUP: 128 gate rows and the same 128 up rows) and
 // output rows per CTA (DOWN: two tiles of 128).
 constexpr int kTcGateUpFeat = kTcRowsA;

@@ -347,8 +347,9 @@ cudaError_t launch(KernelT kern, dim3 grid, size_t smem, cudaStream_t s, const A
 }  // namespace
 
 size_t gemv_stage_bytes(int fmt, int klen, int tokens) {
-  const int per = fmt == FMT_INT4_G32 ? stage_floats_per_token<FMT_INT4_G32>(klen)
-                                      : stage_floats_per_token<FMT_INT8_ROW>(klen);
+  // (Q4_K rows stage like INT4 rows: 32-element chunks with sums)
+  const int per = fmt == FMT_INT8_ROW ? stage_floats_per_token<FMT_INT8_ROW>(klen)
+                                      : stage_floats_per_token<FMT_INT4_G32>(klen);
   return (size_t)per * tokens * sizeof(float);
 }
 

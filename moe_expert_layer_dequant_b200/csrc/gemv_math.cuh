@@ -71,10 +71,35 @@ struct Codes<FMT_INT8_ROW> {
   }
 };
 
+// Q4_K: a chunk is one 32-weight sub-block, staged in natural order. A code
+// run of 32 bytes holds two sub-blocks (low nibbles: weights 4w..4w+3 of
+// word w of the first, high nibbles: of the second), so each nibble half of a
+// word meets four consecutive staged values.
+template <>
+struct Codes<FMT_Q4K> {
+  static constexpr int kChunk = 32;
+  static constexpr int kStageBytes = 80;  // 64 bytes of int16 + 16 bytes pad
+  static __device__ __forceinline__ int slot_of(int j) { return j; }
+  // Words w0, w1 (codes 8h..8h+7 of both sub-blocks) with the staged values
+  // 8h..8h+7 of the low (xl) and high (xh) sub-block.
+  static __device__ __forceinline__ void dot_words(uint32_t w0, uint32_t w1, uint4 xl, uint4 xh, int& pl, int& ph) {
+    const uint32_t l0 = w0 & 0x0F0F0F0Fu, h0 = (w0 >> 4) & 0x0F0F0F0Fu;
+    const uint32_t l1 = w1 & 0x0F0F0F0Fu, h1 = (w1 >> 4) & 0x0F0F0F0Fu;
+    pl = dp2a_lo_u((int)xl.x, l0, pl);
+    pl = dp2a_hi_u((int)xl.y, l0, pl);
+    pl = dp2a_lo_u((int)xl.z, l1, pl);
+    pl = dp2a_hi_u((int)xl.w, l1, pl);
+    ph = dp2a_lo_u((int)xh.x, h0, ph);
+    ph = dp2a_hi_u((int)xh.y, h0, ph);
+    ph = dp2a_lo_u((int)xh.z, h1, ph);
+    ph = dp2a_hi_u((int)xh.w, h1, ph);
+  }
+};
+
 // Stages one chunk of a bf16 activation row (p: the chunk's first element,
 // 16-byte aligned; null for a zero pad row): the int16 values in code order
-// at dst, the chunk's power-of-two factor in *xf and (INT4) its plain sum in
-// *xsum, the sum the min term of the affine format multiplies. With `wn`
+// at dst, the chunk's power-of-two factor in *xf and (INT4, Q4_K) its plain
+// sum in *xsum, the sum the min term of the affine formats multiplies. With `wn`
 // (the same chunk of an RMSNorm weight) the chunk is first normalized:
 // x -> bf16(x * inv_rms * w).
 template <int FMT>
@@ -142,7 +167,7 @@ __device__ __forceinline__ void stage_chunk(const uint16_t* p, uint8_t* dst, flo
     }
     *xf = amax > 0.f ? ldexpf(1.0f, e - 14) : 0.f;
   }
-  if (FMT == FMT_INT4_G32) *xsum = sum;
+  if (FMT == FMT_INT4_G32 || FMT == FMT_Q4K) *xsum = sum;
 }
 
 // Exact int32 dot products of one chunk of codes (wv: 16 bytes) with the

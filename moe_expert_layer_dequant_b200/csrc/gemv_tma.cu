@@ -69,6 +69,8 @@ template <int FMT, int MT, int NM, int NC, int G>
 __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_constant__ TmaGemvArgs a) {
   using C = Codes<FMT>;
   constexpr bool kInt4 = (FMT == FMT_INT4_G32);
+  constexpr bool kQ4K = (FMT == FMT_Q4K);
+  constexpr bool kAffine = kInt4 || kQ4K;   // a min term: staged chunk sums needed
   constexpr int R = NC;  // rows per stage
   extern __shared__ __align__(128) uint8_t smem[];
 
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   // (ks_len) with tensor maps, the slice itself with 1-D copies.
   const int S = a.stages;
   const int wid = maps ? a.ks_len : klen;
-  const int cs = kInt4 ? wid / 2 : wid;
+  const int cs = kInt4 ? wid / 2 : kQ4K ? wid / Q4K::kBlock * Q4K::kBytes : wid;
   const int gst = kInt4 ? wid / 32 : 0;
   const int nch = klen / C::kChunk;
   const int tok_stride = nch * C::kStageBytes;   // bytes of staged int16 per token
@@ -111,8 +113,8 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   uint64_t* empty = full + S;
   uint8_t* xi = smem + 128;                                         // [tok_rows][nch] chunks
   float* xf = reinterpret_cast<float*>(xi + (size_t)tok_rows * tok_stride);  // [tok_rows][nch] factors
-  float* xsum = xf + (size_t)tok_rows * nch;                        // [tok_rows][nch] (INT4)
-  const size_t x_bytes = ((size_t)tok_rows * (tok_stride + 4 * nch + (kInt4 ? 4 * nch : 0)) + 127) / 128 * 128;
+  float* xsum = xf + (size_t)tok_rows * nch;                        // [tok_rows][nch] (INT4, Q4_K)
+  const size_t x_bytes = ((size_t)tok_rows * (tok_stride + 4 * nch + (kAffine ? 4 * nch : 0)) + 127) / 128 * 128;
   // then the input norm's scratch (gemv_norm_bytes)
   uint8_t* stage0 = smem + 128 + x_bytes + gemv_norm_bytes(NC * G);
   const size_t stage_bytes = (size_t)NM * R * (cs + 4 * gst);
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   const int row_stages = (r1 - r0 + R - 1) / R;
   const int tok_blocks = (job.ntok + a.stage_tokens - 1) / a.stage_tokens;
   const int total = row_stages * tok_blocks;
-  const int row_bytes = kInt4 ? job.K / 2 : job.K;
+  const int row_bytes = kInt4 ? job.K / 2 : kQ4K ? job.K / Q4K::kBlock * Q4K::kBytes : job.K;
   const int row_groups = job.K / 32;
 
   // The next kernel in the stream may be scheduled now; it waits for this
@@ -155,7 +157,9 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
           mbar_arrive_expect_tx(&full[slot], (uint32_t)stage_bytes);
 #pragma unroll
           for (int i = 0; i < NM; ++i) {
-            tma_load_2d(st + (size_t)i * R * cs, &jm[i].codes, kInt4 ? k0 / 16 : k0 / 8, n0, &full[slot]);
+            // x in 8-byte elements: 16 INT4 codes, 8 INT8 codes, or 18 per Q4_K block
+            tma_load_2d(st + (size_t)i * R * cs, &jm[i].codes, kInt4 ? k0 / 16 : kQ4K ? k0 / Q4K::kBlock * 18 : k0 / 8,
+                        n0, &full[slot]);
             if (kInt4) {
               tma_load_2d(dsc + (size_t)i * R * gst * 2, &jm[i].scale, k0 / 32, n0, &full[slot]);
               tma_load_2d(dmn + (size_t)i * R * gst * 2, &jm[i].mn, k0 / 32, n0, &full[slot]);
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
       const int slot = s % S, use = s / S;
       const int n = r0 + rs * R + wr;
       float row_scale[NM];
-      if (!kInt4 && n < r1) {
+      if (FMT == FMT_INT8_ROW && n < r1) {
 #pragma unroll
         for (int i = 0; i < NM; ++i) row_scale[i] = __half2float(__ldg(job.m[i].scale + n));
       }
@@ -260,6 +264,60 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
           for (int i = 0; i < NM; ++i)
 #pragma unroll
             for (int t = 0; t < MT; ++t) acc[i][t] = 0.f;
+          if (kQ4K) {
+            // A lane takes code runs u = lane, lane + 32, ...: run u % 4 of
+            // block u / 4 (32 code bytes, two sub-blocks), whose scales and
+            // mins come from the block's 16-byte header.
+            const int nu = klen / 64;
+            for (int u = lane; u < nu; u += 32) {
+              const int bo = (u >> 2) * Q4K::kBytes;
+              const int ox = tc * tok_stride + 2 * u * C::kStageBytes;
+              const int of = tc * nch + 2 * u;
+              uint4 c0[NM], c1[NM];
+#pragma unroll
+              for (int i = 0; i < NM; ++i) {
+                const uint8_t* rb = st + (i * R + wr) * cs + bo + 16 + 32 * (u & 3);
+                c0[i] = *reinterpret_cast<const uint4*>(rb);
+                c1[i] = *reinterpret_cast<const uint4*>(rb + 16);
+              }
+              int pl[NM][MT], ph[NM][MT];
+#pragma unroll
+              for (int t = 0; t < MT; ++t) {
+                const uint8_t* xl = xi + ox + t * tok_stride;
+                const uint8_t* xh = xl + C::kStageBytes;
+#pragma unroll
+                for (int i = 0; i < NM; ++i) pl[i][t] = ph[i][t] = 0;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  const uint4 a = *reinterpret_cast<const uint4*>(xl + 16 * h);
+                  const uint4 b = *reinterpret_cast<const uint4*>(xh + 16 * h);
+#pragma unroll
+                  for (int i = 0; i < NM; ++i) {
+                    const uint4& cw = h < 2 ? c0[i] : c1[i];
+                    const uint32_t w0 = (h & 1) ? cw.z : cw.x, w1 = (h & 1) ? cw.w : cw.y;
+                    Codes<FMT_Q4K>::dot_words(w0, w1, a, b, pl[i][t], ph[i][t]);
+                  }
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < NM; ++i) {
+                const uint4 hdr = *reinterpret_cast<const uint4*>(st + (i * R + wr) * cs + bo);
+                float sl, ml, sh, mh;
+                Q4K::scale_min(hdr, 2 * (u & 3), sl, ml);
+                Q4K::scale_min(hdr, 2 * (u & 3) + 1, sh, mh);
+#pragma unroll
+                for (int t = 0; t < MT; ++t) {
+                  const float fl = xf[of + t * nch], fh = xf[of + 1 + t * nch];
+                  const float Xl = xsum[of + t * nch], Xh = xsum[of + 1 + t * nch];
+                  // sum over both sub-blocks of (d sc q - dmin m) x
+                  float v = fmaf(ml, Xl, acc[i][t]);
+                  v = fmaf(sl * fl, (float)pl[i][t], v);
+                  v = fmaf(mh, Xh, v);
+                  acc[i][t] = fmaf(sh * fh, (float)ph[i][t], v);
+                }
+              }
+            }
+          } else {
           int ox = tc * tok_stride + lane * C::kStageBytes;   // staged activations
           int of = tc * nch + lane;                            // factors / sums
           int oc = 0, og = 0;                                  // code / scale advance
@@ -318,6 +376,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
               }
             }
           }
+          }
           // epilogue
 #pragma unroll
           for (int t = 0; t < MT; ++t) {
@@ -325,7 +384,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
 #pragma unroll
             for (int i = 0; i < NM; ++i) {
               v[i] = warp_sum(acc[i][t]);
-              if (!kInt4) v[i] *= row_scale[i];
+              if (FMT == FMT_INT8_ROW) v[i] *= row_scale[i];
             }
             const int tok = tb + tc + t;
             if (lane == 0 && tok < tn + tb) {
@@ -396,18 +455,22 @@ cudaError_t launch_fmt(const TmaGemvArgs& a, int mt, dim3 grid, size_t smem, cud
 size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
 
 size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages) {
-  const bool i4 = fmt == FMT_INT4_G32;
+  const bool affine = fmt == FMT_INT4_G32 || fmt == FMT_Q4K;   // staged chunk sums
   const size_t red = gemv_norm_bytes(kTmaConsumers * tma_groups(fmt, nm));
-  const int nch = klen / (i4 ? 32 : 16);
-  const int cbytes = i4 ? Codes<FMT_INT4_G32>::kStageBytes : Codes<FMT_INT8_ROW>::kStageBytes;
+  const int nch = klen / (fmt == FMT_INT8_ROW ? 16 : 32);
+  const int cbytes = fmt == FMT_INT8_ROW ? Codes<FMT_INT8_ROW>::kStageBytes : Codes<FMT_INT4_G32>::kStageBytes;
   const int tok_rows = (stage_tokens + mt - 1) / mt * mt;
-  const size_t x_bytes = ((size_t)tok_rows * ((size_t)nch * cbytes + 4 * nch + (i4 ? 4 * nch : 0)) + 127) / 128 * 128;
+  const size_t x_bytes =
+      ((size_t)tok_rows * ((size_t)nch * cbytes + 4 * nch + (affine ? 4 * nch : 0)) + 127) / 128 * 128;
   return 128 + x_bytes + red + tma_gemv_stage_bytes(fmt, nm, klen) * stages;
 }
 
 size_t tma_gemv_stage_bytes(int fmt, int nm, int klen) {
-  const bool i4 = fmt == FMT_INT4_G32;
-  return (size_t)nm * kTmaConsumers * ((i4 ? klen / 2 : klen) + 4 * (i4 ? klen / 32 : 0));
+  size_t row;
+  if (fmt == FMT_INT4_G32) row = klen / 2 + 4 * (klen / 32);   // codes, scales, mins
+  else if (fmt == FMT_Q4K) row = (size_t)klen / Q4K::kBlock * Q4K::kBytes;
+  else row = klen;
+  return (size_t)nm * kTmaConsumers * row;
 }
 
 cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, int jobs, cudaStream_t s) {
@@ -415,6 +478,8 @@ cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, in
   const dim3 grid(a.ctas_per_job, splits, jobs);
   if (a.fmt == FMT_INT4_G32)
     return nm == 2 ? launch_fmt<FMT_INT4_G32, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_INT4_G32, 1>(a, mt, grid, smem, s);
+  if (a.fmt == FMT_Q4K)
+    return nm == 2 ? launch_fmt<FMT_Q4K, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_Q4K, 1>(a, mt, grid, smem, s);
   return nm == 2 ? launch_fmt<FMT_INT8_ROW, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_INT8_ROW, 1>(a, mt, grid, smem, s);
 }
 
@@ -427,6 +492,13 @@ cudaError_t encode_qw_maps(QWMaps* m, int fmt, const QW& w, int N, int K, int ks
     e = encode_tmap_2d(&m->scale, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.scale, K / 32, N, K / 16, ks_len / 32, R);
     if (e != cudaSuccess) return e;
     return encode_tmap_2d(&m->mn, CU_TENSOR_MAP_DATA_TYPE_UINT16, w.mn, K / 32, N, K / 16, ks_len / 32, R);
+  }
+  if (fmt == FMT_Q4K) {   // 18 eight-byte elements per block; the boxes hold whole blocks
+    e = encode_tmap_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT64, w.q, K / Q4K::kBlock * 18, N,
+                       (size_t)K / Q4K::kBlock * Q4K::kBytes, ks_len / Q4K::kBlock * 18, R);
+    m->scale = m->codes;
+    m->mn = m->codes;
+    return e;
   }
   e = encode_tmap_2d(&m->codes, CU_TENSOR_MAP_DATA_TYPE_UINT64, w.q, K / 8, N, K, ks_len / 8, R);
   m->scale = m->codes;

@@ -7,11 +7,11 @@
 namespace moeffn {
 
 constexpr int kTmaConsumers = 8;  // consumer warps per group = rows per stage
-// Consumer groups, taking stages in turn: three for a single INT4 matrix (the
-// down projection; more warps to hide the per-stage arithmetic latency), two
+// Consumer groups, taking stages in turn: three for a single INT4 or Q4_K
+// matrix (the down projection; more warps to hide the per-stage arithmetic latency), two
 // otherwise (the fused gate/up pair's larger stages leave room for fewer slots,
 // and the INT8 consumers need more registers than 800 threads allow).
-constexpr int tma_groups(int fmt, int nm) { return (nm == 1 && fmt == FMT_INT4_G32) ? 3 : 2; }
+constexpr int tma_groups(int fmt, int nm) { return (nm == 1 && (fmt == FMT_INT4_G32 || fmt == FMT_Q4K)) ? 3 : 2; }
 // Token rows whose input norm the GEMV's staging applies (more: a norm launch first).
 constexpr int kGemvNormTokens = 8;
 // Shared memory of the staging's input-norm pass: inverse RMS per staged token
@@ -20,7 +20,8 @@ __host__ __device__ constexpr size_t gemv_norm_bytes(int consumer_warps) {
   return ((size_t)kGemvNormTokens * (1 + consumer_warps) * 4 + 127) / 128 * 128;
 }
 
-// Tensor maps of one K-split matrix: codes (u64 elements), scales, mins (u16).
+// Tensor maps of one K-split matrix: codes (u64 elements), scales, mins (u16;
+// INT4 only).
 struct QWMaps {
   CUtensorMap codes, scale, mn;
 };
@@ -59,7 +60,7 @@ struct TmaGemvArgs {
                                // of each row range (null: fp32 partials only, a tail kernel adds them)
   const uint16_t* norm_w;      // dense gate/up, unsplit K: normalize x on staging (RMSNorm weight [K]), or null
   float eps;
-  int ks_len;                  // K elements per split (INT4: multiple of 256)
+  int ks_len;                  // K elements per split (INT4, Q4_K: multiple of 256)
   int ctas_per_job;
   int stage_tokens;
   int stages;

@@ -42,11 +42,45 @@ __global__ void k_dequant(const QW w, int fmt, int N, int K, float* out_f32, uin
   }
 }
 
+// Q4_K: one thread per code word (4 bytes of a run): weights 64c + 4v .. + 3
+// of the low sub-block and the same + 32 of the high one, each
+// fmaf(q, d * scale, -dmin * min) as in the GEMV and GEMM.
+__global__ void k_dequant_q4k(const uint8_t* q, int N, int K, float* out_f32, uint16_t* out_bf16) {
+  const size_t words = (size_t)N * (K / Q4K::kBlock) * 32;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < words; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t blk = i / 32;                   // block index over the whole matrix
+    const int v = (int)(i % 32), c = v / 8;      // word v of the block's codes, in run c
+    const uint8_t* b = q + blk * Q4K::kBytes;
+    const uint4 hdr = *reinterpret_cast<const uint4*>(b);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(b + 16 + 4 * v);
+    float sl, ml, sh, mh;
+    Q4K::scale_min(hdr, 2 * c, sl, ml);
+    Q4K::scale_min(hdr, 2 * c + 1, sh, mh);
+    const size_t e0 = blk * Q4K::kBlock + 64 * c + 4 * (v % 8);   // element index (row-major: blocks in order)
+    for (int j = 0; j < 4; ++j) {
+      const float lo = fmaf((float)((w >> (8 * j)) & 15u), sl, ml);
+      const float hi = fmaf((float)((w >> (8 * j + 4)) & 15u), sh, mh);
+      if (out_f32) { out_f32[e0 + j] = lo; out_f32[e0 + 32 + j] = hi; }
+      if (out_bf16) { out_bf16[e0 + j] = float_to_bf16_bits(lo); out_bf16[e0 + 32 + j] = float_to_bf16_bits(hi); }
+    }
+  }
+}
+
 }  // namespace
 
 extern "C" {
 
 int moeffn_test_dequant(const moeffn_qweight* w, float* out_f32, uint16_t* out_bf16, moeffn_stream_t stream) {
+  if (w != nullptr && w->format == MOEFFN_Q_Q4_K) {
+    if (w->q == nullptr) return api_fail(MOEFFN_ERR_INVALID, "test_dequant: null");
+    if (w->rows < 1 || w->cols < 256 || w->cols % 256 != 0) return api_fail(MOEFFN_ERR_INVALID, "test_dequant: shape");
+    if ((reinterpret_cast<uintptr_t>(w->q) & 15u) != 0) return api_fail(MOEFFN_ERR_INVALID, "test_dequant: q misaligned");
+    k_dequant_q4k<<<296, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<const uint8_t*>(w->q), w->rows,
+                                                                          w->cols, out_f32, out_bf16);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return api_fail(MOEFFN_ERR_CUDA, cudaGetErrorString(e));
+    return MOEFFN_OK;
+  }
   if (w == nullptr || w->q == nullptr || w->scale == nullptr) return api_fail(MOEFFN_ERR_INVALID, "test_dequant: null");
   if (w->format != MOEFFN_Q_INT8_ROW && w->format != MOEFFN_Q_INT4_AFFINE_G32)
     return api_fail(MOEFFN_ERR_UNSUPPORTED, "test_dequant: format");

@@ -40,6 +40,11 @@ design notes of the repository):
    activation, the FFN output before a tail, the shared-expert output, the
    seed, the routed output ``y`` and the layer output. Router logits and the
    shared-expert gate logit are fp32; gate/up/down dot products are float64.
+7. The K-quant block type Q4_K ([llama]: a Q4_K_M file mixes block types per
+   tensor, resolved by ``encode_gemv_any``) is not laid out on the pages; its
+   layout is the public GGUF one (256-weight super-blocks of 144 bytes: fp16 d
+   and dmin, eight 6-bit scales and mins packed in 12 bytes, 128 bytes of
+   4-bit codes), with w = d * scale * q - dmin * min rounded once to fp32.
 """
 from __future__ import annotations
 
@@ -128,12 +133,74 @@ def dequant_int4_affine_g32(packed: np.ndarray, scale: np.ndarray, mn: np.ndarra
     return q * s + m
 
 
+Q4K_BLOCK = 256       # weights per K-quant super-block
+Q4K_BYTES = 144       # 2 (d) + 2 (dmin) + 12 (packed 6-bit scales and mins) + 128 (codes)
+
+
+def q4_k_scales_mins(packed12: np.ndarray):
+    """The eight 6-bit (scale, min) pairs of a Q4_K super-block from its 12
+    packed bytes [..., 12] (the GGUF K-quant layout, which the pages name as
+    the block type of a Q4_K_M file but do not spell out, reading 7):
+
+    * sub-blocks 0..3: scale = low 6 bits of byte j, min = low 6 bits of byte j + 4;
+    * sub-blocks 4..7: the low 4 bits of scale and min are the low and high
+      nibble of byte j + 4, and their top 2 bits are the top 2 bits of bytes
+      j - 4 (scale) and j (min).
+    """
+    b = np.asarray(packed12, np.int64)
+    sc = np.empty(b.shape[:-1] + (8,), np.int64)
+    mn = np.empty_like(sc)
+    for j in range(4):
+        sc[..., j] = b[..., j] & 63
+        mn[..., j] = b[..., j + 4] & 63
+    for j in range(4, 8):
+        sc[..., j] = (b[..., j + 4] & 15) | ((b[..., j - 4] >> 6) << 4)
+        mn[..., j] = (b[..., j + 4] >> 4) | ((b[..., j] >> 6) << 4)
+    return sc, mn
+
+
+def q4_k_codes(blocks: np.ndarray) -> np.ndarray:
+    """Codes [..., 256] of super-blocks [..., 144]: the 128 code bytes are four
+    runs of 32; run c holds elements 64c..64c+31 in its low nibbles and
+    64c+32..64c+63 in its high nibbles."""
+    qs = np.asarray(blocks, np.int64)[..., 16:Q4K_BYTES]
+    q = np.empty(qs.shape[:-1] + (Q4K_BLOCK,), np.int64)
+    for c in range(4):
+        run = qs[..., 32 * c:32 * c + 32]
+        q[..., 64 * c:64 * c + 32] = run & 15
+        q[..., 64 * c + 32:64 * c + 64] = run >> 4
+    return q
+
+
+def dequant_q4_k(blocks: np.ndarray, N: int, K: int) -> np.ndarray:
+    """W[n][k] of a Q4_K matrix stored as super-blocks [N][K/256][144]:
+    w = d * scale_j * q - dmin * min_j for element k of sub-block j = (k % 256) // 32,
+    with d and dmin the block's fp16 super-scales (little-endian bytes 0-1, 2-3).
+
+    Both products are exact in fp32 (at most 21 and 17 significant bits), so
+    the value is the exact difference rounded once to fp32, which is what the
+    format's fp32 dequantization gives with or without a fused multiply-add
+    (reading 7). The difference is formed exactly in float64 whenever its
+    fp32 rounding depends on it.
+    """
+    b = np.asarray(blocks, np.uint8).reshape(N, K // Q4K_BLOCK, Q4K_BYTES)
+    d = b[..., 0:2].copy().view(np.float16)[..., 0].astype(np.float64)
+    dmin = b[..., 2:4].copy().view(np.float16)[..., 0].astype(np.float64)
+    sc, mn = q4_k_scales_mins(b[..., 4:16])
+    q = q4_k_codes(b)
+    sub = np.arange(Q4K_BLOCK) // 32
+    w = d[..., None] * sc[..., sub] * q - dmin[..., None] * mn[..., sub]
+    return f32(w).reshape(N, K)
+
+
 def dequant(w) -> np.ndarray:
     """Dequantize a ``synth.QWeight``-like object (fields fmt, q, scale, min)."""
     if w.fmt == "int8_row":
         return dequant_int8_row(w.q, w.scale)
     if w.fmt == "int4_g32":
         return dequant_int4_affine_g32(w.q, w.scale, w.min)
+    if w.fmt == "q4_k":
+        return dequant_q4_k(w.q, w.N, w.K)
     raise ValueError(f"unknown format {w.fmt}")
 
 

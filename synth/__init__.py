@@ -34,6 +34,7 @@ import torch
 
 FMT_INT8_ROW = "int8_row"
 FMT_INT4_G32 = "int4_g32"
+FMT_Q4_K = "q4_k"      # GGUF K-quant super-blocks: 256 weights in 144 bytes
 
 # Tensor ids of the random streams.
 _T_X, _T_RES, _T_NORM_W, _T_ROUTER, _T_WSG = 0, 1, 2, 3, 4
@@ -94,13 +95,14 @@ class QWeight:
     fmt: str
     N: int
     K: int
-    q: np.ndarray                    # int8 [N][K] or uint8 packed [N][K/2]
-    scale: np.ndarray                # fp16 [N] or [N][K/32]
+    q: np.ndarray                    # int8 [N][K], uint8 packed [N][K/2] or Q4_K blocks [N][K/256*144]
+    scale: Optional[np.ndarray]      # fp16 [N] or [N][K/32]; None for Q4_K (in the blocks)
     min: Optional[np.ndarray] = None  # fp16 [N][K/32] (INT4 only)
 
     @property
     def nbytes(self) -> int:
-        return int(self.q.nbytes + self.scale.nbytes + (0 if self.min is None else self.min.nbytes))
+        return int(self.q.nbytes + (0 if self.scale is None else self.scale.nbytes)
+                   + (0 if self.min is None else self.min.nbytes))
 
 
 @dataclass
@@ -128,6 +130,19 @@ def random_qweight(fmt: str, N: int, K: int, rng: np.random.Generator,
         scale = rng.uniform(*int4_scale, size=(N, K // 32)).astype(np.float16)
         mn = rng.normal(0.0, int4_min_sd, size=(N, K // 32)).astype(np.float16)
         return QWeight(fmt, N, K, packed, scale, mn)
+    if fmt == FMT_Q4_K:
+        if K % 256:
+            raise ValueError("Q4_K needs K % 256 == 0")
+        nb = K // 256
+        # Effective step d * scale in [0, 0.04) and offset dmin * min in
+        # [0, 0.13), the ranges of the INT4-affine weights; the packed scale
+        # bytes and the codes are uniform bytes (every 6-bit field uniform).
+        blocks = rng.integers(0, 256, size=(N, nb, 144), dtype=np.uint8)
+        d = rng.uniform(int4_scale[0] / 32, int4_scale[1] / 32, size=(N, nb)).astype(np.float16)
+        dmin = rng.uniform(0.0005, 0.002, size=(N, nb)).astype(np.float16)
+        blocks[..., 0:2] = d.view(np.uint8).reshape(N, nb, 2)
+        blocks[..., 2:4] = dmin.view(np.uint8).reshape(N, nb, 2)
+        return QWeight(fmt, N, K, blocks.reshape(N, nb * 144), None)
     raise ValueError(f"unknown format {fmt}")
 
 
@@ -209,6 +224,8 @@ def zero_like_qweight(fmt: str, N: int, K: int) -> QWeight:
     """An all-zero matrix (q = 0, scale = 0, min = 0) for hand-built cases."""
     if fmt == FMT_INT8_ROW:
         return QWeight(fmt, N, K, np.zeros((N, K), np.int8), np.zeros(N, np.float16))
+    if fmt == FMT_Q4_K:
+        return QWeight(fmt, N, K, np.zeros((N, K // 256 * 144), np.uint8), None)
     return QWeight(fmt, N, K, np.zeros((N, K // 2), np.uint8), np.zeros((N, K // 32), np.float16),
                    np.zeros((N, K // 32), np.float16))
 

@@ -86,6 +86,12 @@ def test_refusals_before_launch():
     mixed.up = _fake_qweight(lib, lib.Q_INT8_ROW, 512, 256, 0x30000000)
     assert L.ffn_dense(ctypes.byref(mixed), x, r, 2, 0, ws, 1 << 30, None) == -2
     assert b"gate and up" in L.moeffn_last_error()
+    q4k = _fake_ffn(lib, lib.Q_Q4_K, 256 + 128, 512)                                 # Q4_K: K % 256 != 0
+    assert L.ffn_dense(ctypes.byref(q4k), x, r, 2, 0, ws, 1 << 30, None) == -1
+    assert b"256" in L.moeffn_last_error()
+    q4k = _fake_ffn(lib, lib.Q_Q4_K, 256, 512)
+    q4k.gate.q = 0x10000008                                                          # misaligned blocks
+    assert L.ffn_dense(ctypes.byref(q4k), x, r, 2, 0, ws, 1 << 30, None) == -1
     shape = _fake_ffn(lib, lib.Q_INT8_ROW, 256, 512)
     shape.down = _fake_qweight(lib, lib.Q_INT8_ROW, 512, 256, 0x30000000)           # transposed down
     assert L.ffn_dense(ctypes.byref(shape), x, r, 2, 0, ws, 1 << 30, None) == -1
@@ -110,6 +116,8 @@ def test_router_and_plan_refusals():
     h = ctypes.c_void_p()
     assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -2
     assert b"INT4" in L.moeffn_last_error()
+    q4k_experts = (lib._FFN * 8)(*[_fake_ffn(lib, lib.Q_Q4_K, 256, 512) for _ in range(8)])
+    assert L.moe_plan_create(ctypes.byref(lib._MoeDesc(8, 2, 0, router, q4k_experts, None, None)), ctypes.byref(h)) == -2
     desc.top_k = 0
     assert L.moe_plan_create(ctypes.byref(desc), ctypes.byref(h)) == -2
     assert L.moe_layer(None, x, 0x50000000, 1, None, ws, 1 << 20, None) == -1

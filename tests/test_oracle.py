@@ -50,6 +50,57 @@ def test_dequant_int4_subnormal_scale_exact():
     assert np.array_equal(oracle.dequant_int4_affine_g32(packed, scale, mn)[0], want)
 
 
+def _q4k_block(header_bytes, codes):
+    return np.concatenate([np.asarray(header_bytes, np.uint8), np.asarray(codes, np.uint8)])[None, :]
+
+
+def test_dequant_q4_k_golden_block():
+    """Hand-derived Q4_K super-block (golden q4_k_block.txt): the 6-bit
+    scale/min unpacking of all eight sub-blocks and values in each of them."""
+    kv, _ = read_golden("q4_k_block.txt")
+    header = [int(t, 16) for t in kv["header_hex"]]
+    assert kv["codes"] == ["0..127"]
+    blk = _q4k_block(header, np.arange(128))
+    sc, mn = oracle.q4_k_scales_mins(blk[0, 4:16])
+    want = [tuple(int(v) for v in t.split(",")) for t in kv["scales_mins"]]
+    assert list(zip(sc.tolist(), mn.tolist())) == want
+    w = oracle.dequant_q4_k(blk, 1, 256)[0]
+    for t in kv["expected"]:
+        k, v = t.split(":")
+        assert w[int(k)] == float(v), (k, w[int(k)], v)
+
+
+@pytest.mark.parametrize("c,r,hi", [(0, 0, False), (0, 31, True), (1, 7, False), (2, 16, True), (3, 31, False),
+                                   (3, 31, True)])
+def test_q4_k_code_runs(c, r, hi):
+    """One code of 1 in byte r of run c (low or high nibble), all scales 1,
+    mins 0, d = 1: exactly element 64c + r (+ 32 for the high nibble) is 1."""
+    header = [0x00, 0x3C, 0, 0] + [1, 1, 1, 1, 0, 0, 0, 0, 1, 1, 1, 1]   # d = 1, dmin = 0, scale 1, min 0
+    codes = np.zeros(128, np.uint8)
+    codes[32 * c + r] = 0x10 if hi else 0x01
+    w = oracle.dequant_q4_k(_q4k_block(header, codes), 1, 256)[0]
+    want = np.zeros(256)
+    want[64 * c + r + (32 if hi else 0)] = 1.0
+    assert np.array_equal(w, want)
+
+
+def test_q4_k_rounds_once_to_fp32():
+    """d * scale * q is exact; the difference with dmin * min is rounded once
+    to fp32, ties to even: 945 - 2^-15 lies halfway between 945 - 2^-14 and 945
+    (fp32 spacing 2^-14 there) and rounds to 945 (even significand);
+    945 - 3 * 2^-15 lies halfway between 945 - 2^-14 (odd) and 945 - 2^-13
+    (even) and rounds to the latter; zero blocks give zeros."""
+    def one(dmin_bits, m):
+        # d = 1, scale 63 for sub-block 0, min m, codes 15
+        s = [63, 0, 0, 0, m, 0, 0, 0, 0, 0, 0, 0]
+        header = [0x00, 0x3C, dmin_bits & 0xFF, dmin_bits >> 8] + s
+        return oracle.dequant_q4_k(_q4k_block(header, np.full(128, 0xFF, np.uint8)), 1, 256)[0, 0]
+    half_ulp = 0x0200   # fp16 subnormal 512 * 2^-24 = 2^-15
+    assert one(half_ulp, 1) == 945.0
+    assert one(half_ulp, 3) == 945.0 - 2.0 ** -13
+    assert np.all(oracle.dequant_q4_k(np.zeros((2, 288), np.uint8), 2, 512) == 0.0)
+
+
 def test_dequant_int8_golden_block():
     kv, _ = read_golden("int8_row_block.txt")
     q = np.array([[int(t) for t in kv["q_row0"]], [int(t) for t in kv["q_row1"]]], np.int8)
