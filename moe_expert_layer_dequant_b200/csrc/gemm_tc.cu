@@ -19,7 +19,9 @@
 //              A tiles;
 //  warp 1      allocates TMEM; one thread issues tile 0's tcgen05.mma;
 //  warp 2      token producer: TMA loads of the bf16 token tiles (128-byte
-//              swizzled, K = 64 per stage), the MMA's B operand;
+//              swizzled, K = 64 per stage), the MMA's B operand, one per A
+//              stage slot (the two operands of a stage share one full and
+//              one empty barrier);
 //  warp 3      one thread issues tile 1's tcgen05.mma (the two accumulators
 //              are independent; issuing from two threads halves the per-stage
 //              issue time); A and B slots are released once both issuers'
@@ -28,11 +30,15 @@
 //              in turn: a thread owns one weight row of one A tile and turns
 //              the 64 codes of two quantization groups into bf16 (RNE of the
 //              exact fp32 value q * scale + min), stored to its TMEM lane (32
-//              columns of bf16 pairs); then, as the epilogue, read the
-//              accumulators (tcgen05.ld) and write the outputs.
+//              columns of bf16 pairs); one thread per set waits on and
+//              arrives at the mbarriers for the set, whose warps meet at a
+//              named barrier before and after the stage; then, as the
+//              epilogue, read the accumulators (tcgen05.ld) and write the
+//              outputs.
 //
 // TMEM columns: accumulator of A tile t at [t * ntile, (t + 1) * ntile); a ring
-// of A stages (two K groups each: 32 columns per A tile) after them. Waits
+// of A stages (two K groups each: 32 columns per A tile) after them; the
+// ring depth SA (at most 6) is what the accumulators leave. Waits
 // suspend the waiting thread (mbarrier.try_wait) rather than spin, so the
 // producer and MMA threads take no issue slots from the dequantizing warps.
 // Modes: GATEUP writes bf16(act(gate) * up); DOWN writes fp32 partial sums
@@ -52,8 +58,7 @@ constexpr int kTilesA = 2;                   // A tiles per CTA
 constexpr int kDqWarps = 16;                 // warps 4..19, two sets of 8
 constexpr int kThreads = 32 * (4 + kDqWarps);
 constexpr int kSW = 3;                       // quantized weight stages
-constexpr int kSB = 3;                       // token stages (K = 64 each)
-constexpr int kBStageBytes = kTcMaxTok * 128;
+constexpr int kBRingBytes = 64 * 1024;      // token stages: one per A stage slot (SA * ntile * 128 bytes)
 constexpr int kTmemCols = 512;
 constexpr int kAStageCols = 32 * kTilesA;    // two K groups (64 bf16 = 32 columns) per A tile
 
@@ -90,15 +95,13 @@ struct TcFmt<FMT_Q4K> {
 
 template <int FMT>
 constexpr size_t tc_smem_bytes() {
-  return 1024 /*align slack*/ + 1024 /*barriers*/ + (size_t)kSW * TcFmt<FMT>::kStageBytes +
-         (size_t)kSB * kBStageBytes;
+  return 1024 /*align slack*/ + 1024 /*barriers*/ + (size_t)kSW * TcFmt<FMT>::kStageBytes + kBRingBytes;
 }
 static_assert(tc_smem_bytes<FMT_INT4_G32>() <= 232448, "shared memory");
 static_assert(tc_smem_bytes<FMT_INT8_ROW>() <= 232448, "shared memory");
 static_assert(tc_smem_bytes<FMT_Q4K>() <= 232448, "shared memory");
 static_assert(TcFmt<FMT_INT4_G32>::kStageBytes % 1024 == 0 && TcFmt<FMT_INT8_ROW>::kStageBytes % 1024 == 0 &&
-                  TcFmt<FMT_Q4K>::kStageBytes % 1024 == 0 &&
-                  kBStageBytes % 1024 == 0,
+                  TcFmt<FMT_Q4K>::kStageBytes % 1024 == 0,
               "stage bases stay 1024-byte aligned (128-byte swizzle)");
 
 struct Job {
@@ -266,7 +269,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   const int klen = min(a.ks_len, job.K - k0);     // a multiple of the weight stage K
   const int nA = klen / 64;                         // A stages (two K groups each)
   const int nW = klen / F::kKTile;                  // weight stages
-  const int nB = klen / 64;                         // token stages
   const int tn = min(ntile, job.ntok - t0);         // valid token rows
   const int nmma = (tn + 15) & ~15;                 // MMA N
   const int SA = min(8, (kTmemCols - kTilesA * ntile) / kAStageCols) & ~1;   // A ring depth (even)
@@ -278,20 +280,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   uint64_t* bars = reinterpret_cast<uint64_t*>(gbase);
   uint64_t* w_full = bars;
   uint64_t* w_empty = w_full + kSW;
-  uint64_t* b_full = w_empty + kSW;
-  uint64_t* b_empty = b_full + kSB;
-  uint64_t* a_full = b_empty + kSB;
-  uint64_t* a_empty = a_full + 8;
-  uint64_t* acc_full = a_empty + 8;
+  uint64_t* full = w_empty + kSW;     // [8] A stage dequantized and its token tile landed
+  uint64_t* empty = full + 8;         // [8] both MMA issuers done with the slot
+  uint64_t* acc_full = empty + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + 512);
+  volatile int* set_dead = reinterpret_cast<volatile int*>(gbase + 520);   // [2] a set's waiter gave up
   const uint32_t w_base = base + 1024;
   const uint32_t b_base = w_base + kSW * F::kStageBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSW; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], kDqWarps); }
-    for (int i = 0; i < kSB; ++i) { mbar_init(&b_full[i], 1); mbar_init(&b_empty[i], 2); }
-    for (int i = 0; i < 8; ++i) { mbar_init(&a_full[i], kDqWarps / 2); mbar_init(&a_empty[i], 2); }
+    for (int i = 0; i < kSW; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], 2); }
+    // full: one arrival per dequantizing set plus the token producer's
+    // expect_tx arrival (and its bytes); empty: one commit per MMA issuer.
+    for (int i = 0; i < 8; ++i) { mbar_init(&full[i], 2); mbar_init(&empty[i], 2); }
+    set_dead[0] = set_dead[1] = 0;
     mbar_init(acc_full, 2);
     fence_mbar_init();
   }
@@ -338,14 +341,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
     // ---------------- token producer ----------------
     if (lane == 0 && SA >= 2) {
       int issued = 0;
-      for (int b = 0; b < nB; ++b, ++issued) {
-        const int slot = b % kSB, use = b / kSB;
-        if (use > 0 && !mbar_wait(&b_empty[slot], (use - 1) & 1)) break;
-        mbar_arrive_expect_tx(&b_full[slot], (uint32_t)ntile * 128u);
-        uint8_t* dst = gbase + (b_base - base) + slot * kBStageBytes;
-        tma_load_2d(dst, job.xmap, k0 + b * 64, row_tok, &b_full[slot]);
+      for (int b = 0; b < nA; ++b, ++issued) {
+        const int slot = b % SA, use = b / SA;
+        if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[slot], (uint32_t)ntile * 128u);
+        uint8_t* dst = gbase + (b_base - base) + slot * ntile * 128;
+        tma_load_2d(dst, job.xmap, k0 + b * 64, row_tok, &full[slot]);
       }
-      for (int b = max(0, issued - kSB); b < issued; ++b) mbar_wait(&b_full[b % kSB], (b / kSB) & 1);
+      for (int b = max(0, issued - SA); b < issued; ++b) mbar_wait(&full[b % SA], (b / SA) & 1);
     }
   } else if (warp == 1 || warp == 3) {
     // ---------------- MMA issuers: warp 1 for A tile 0, warp 3 for tile 1 ----
@@ -356,11 +359,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
     if (lane == 0 && SA >= 2) {
       const uint32_t idesc = idesc_bf16_f32(kTcRowsA, nmma);
       for (int s = 0; s < nA; ++s) {
-        const int slot = s % SA, bs = s % kSB;
-        if (!mbar_wait(&a_full[slot], (s / SA) & 1)) break;
-        if (!mbar_wait(&b_full[bs], (s / kSB) & 1)) break;
+        const int slot = s % SA;
+        if (!mbar_wait(&full[slot], (s / SA) & 1)) break;
         tc_fence_after();
-        const uint64_t bd = umma_desc_sw128(b_base + bs * kBStageBytes);
+        const uint64_t bd = umma_desc_sw128(b_base + slot * ntile * 128);
         const uint32_t acol = tmem + a_col0 + (uint32_t)(slot * kAStageCols);
         if (tl < tiles) {
 #pragma unroll
@@ -368,8 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
             umma_bf16_ts(tmem + (uint32_t)(tl * ntile), acol + (uint32_t)(tl * 32 + kk * 8), bd + 2 * kk, idesc,
                          (s | kk) != 0);
         }
-        umma_commit(&a_empty[slot]);
-        umma_commit(&b_empty[bs]);
+        umma_commit(&empty[slot]);
       }
       umma_commit(acc_full);
       mbar_wait(acc_full, 0);   // every MMA has completed before TMEM is freed
@@ -380,15 +381,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
     const int set = i >> 3, q = i & 3, t = (i >> 2) & 1;   // K-group parity, lane quarter, A tile
     const int r = 32 * q + lane;                           // weight row of the A tile
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // One thread per set (lane 0 of the set's first warp) waits on the
+    // barriers and arrives for the set; the set's eight warps meet at a named
+    // barrier before and after the dequantization.
+    const bool waiter = (i & 7) == 0 && lane == 0;
     bool dead = SA < 2;
     for (int s = set; s < nA && !dead; s += 2) {
       const int slot = s % SA, use = s / SA;
       constexpr int kAPerW = F::kGroups / 2;                           // A stages per weight stage
       const int w = s / kAPerW, g = 2 * (s % kAPerW), ws = w % kSW;
-      bool ok = true;
-      if (s % kAPerW == set) ok = mbar_wait(&w_full[ws], (w / kSW) & 1);   // first A stage of the weight stage for this set
-      if (ok && use > 0) ok = mbar_wait(&a_empty[slot], (use - 1) & 1);
-      if (__any_sync(0xffffffffu, !ok)) { dead = true; break; }
+      if (waiter) {
+        bool ok = true;
+        if (s % kAPerW == set) ok = mbar_wait(&w_full[ws], (w / kSW) & 1);   // first A stage of the weight stage for this set
+        if (ok && use > 0) ok = mbar_wait(&empty[slot], (use - 1) & 1);
+        if (!ok) set_dead[set] = 1;
+      }
+      named_sync(1 + set, 256);
+      if (set_dead[set] != 0) { dead = true; break; }   // the whole set leaves together
+      tc_fence_after();
       if (t < tiles) {
         uint32_t o0[16], o1[16];
         const uint32_t tile = w_base + ws * F::kStageBytes + t * F::kTileBytes;
@@ -401,9 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
         tmem_wait_st();
       }
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&a_full[slot]);
+      named_sync(1 + set, 256);
+      if (waiter) {
+        mbar_arrive(&full[slot]);
         if (s % kAPerW == kAPerW - 2 + set) mbar_arrive(&w_empty[ws]);   // this set's last A stage of the weight stage
       }
     }
