@@ -408,3 +408,25 @@ def test_workspace_too_small_is_refused():
     with pytest.raises(lib.MoeffnError) as e:
         lib.ffn_dense(dl.ffn, dev_bf16(inp.x), dev_bf16(inp.residual), "silu", ws=ws)
     assert e.value.status == -3
+
+
+def test_one_plan_serves_a_sequence_of_token_counts():
+    """One plan and one weight set called with a sequence of token counts that
+    crosses the GEMV / tensor-core switch (8 rows) and back: every call stays
+    at parity with the oracle, top-k indices included (where the oracle's
+    k-th / (k+1)-th logit margin is clear), and no fault is recorded (the
+    routing's arrival counter is reset for every call)."""
+    c = synth.scaled_config(4, H=256, I=256, E=16, k=4, I_s=256)
+    w = synth.make_weights(c, 12)
+    dl = None
+    for M in (3, 40, 1, 64, 65, 7, 9):
+        inp = synth.make_inputs(c, M, 12, weights=w)
+        if dl is None:
+            dl = DeviceLayer(inp)
+        out, idx = dl.run(inp.x, inp.residual, topk_out=True)
+        want, it = oracle.moe_layer(inp, return_internals=True)
+        assert_bf16_close(out, want, f"out M={M}")
+        lg = np.sort(it["logits"], axis=1)[:, ::-1]           # the oracle's k-th / (k+1)-th margin
+        clear = lg[:, c.k - 1] - lg[:, c.k] > 1e-4 * np.sqrt(np.mean(it["logits"] ** 2))
+        assert np.array_equal(idx[clear], it["idx"][clear]), M
+    assert lib.device_faults(True) == 0
