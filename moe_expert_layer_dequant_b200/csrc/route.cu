@@ -208,15 +208,29 @@ __device__ void place_pairs(const RouteArgs& a, int* sm) {
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
+    // Exclusive prefix of the counts and the ascending union, 32 experts at a
+    // time: a warp scan of the counts and a ballot of the nonzero ones.
     int acc = 0, nu = 0;
-    for (int e = 0; e < E; ++e) {
-      offs[e] = acc;
-      acc += counts[e];
-      if (counts[e] > 0 && a.union_list != nullptr) a.union_list[nu++] = e;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int cnt = e < E ? counts[e] : 0;
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (e < E) offs[e] = acc + incl - cnt;
+      const unsigned nz = __ballot_sync(0xffffffffu, cnt > 0);
+      if (cnt > 0 && a.union_list != nullptr) a.union_list[nu + __popc(nz & ((1u << lane) - 1u))] = e;
+      acc += __shfl_sync(0xffffffffu, incl, 31);
+      nu += __popc(nz);
     }
-    offs[E] = acc;
-    if (a.n_union != nullptr) *a.n_union = nu;
+    if (lane == 0) {
+      offs[E] = acc;
+      if (a.n_union != nullptr) *a.n_union = nu;
+    }
   }
   __syncthreads();
   for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = offs[e];

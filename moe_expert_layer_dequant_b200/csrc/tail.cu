@@ -27,6 +27,7 @@ namespace moeffn {
 
 namespace {
 
+
 __device__ __forceinline__ float sum_splits(const float* d, int splits, size_t split_stride, size_t off) {
   float h = 0.f;
   for (int s = 0; s < splits; ++s) h += d[s * split_stride + off];   // fixed split order
@@ -34,6 +35,8 @@ __device__ __forceinline__ float sum_splits(const float* d, int splits, size_t s
 }
 
 // Four consecutive features per thread (16-byte partial loads); N % 4 == 0.
+// KMAX: a bound on top-k (2, 4, 8 or 16), so that the per-rank registers stay few.
+template <int KMAX>
 __global__ void k_tail_elementwise(const TailArgs a) {
   pdl_launch_dependents();
   pdl_wait();
@@ -62,16 +65,32 @@ __global__ void k_tail_elementwise(const TailArgs a) {
         acc[0] = round_bf16(round_bf16(sh.x) * g); acc[1] = round_bf16(round_bf16(sh.y) * g);
         acc[2] = round_bf16(round_bf16(sh.z) * g); acc[3] = round_bf16(round_bf16(sh.w) * g);
       }
-      for (int r = 0; r < a.k; ++r) {   // seed first, then the ranks in order
-        const int slot = a.inv[t * a.k + r];
-        const float wr = a.w[t * a.k + r];
-        float4 d = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp = 0; sp < a.splits; ++sp) {
-          const float4 v = *reinterpret_cast<const float4*>(a.d + sp * rstride + (size_t)slot * a.N + n);
-          d.x += v.x; d.y += v.y; d.z += v.z; d.w += v.w;
+      // All ranks' slots and weights first, then every rank's partials split
+      // by split (the loads of one split are independent), then the sum:
+      // seed first, then the ranks in order; each rank's splits in order.
+      int slot[KMAX];
+      float wr[KMAX];
+      float4 d[KMAX];
+#pragma unroll
+      for (int r = 0; r < KMAX; ++r) {
+        d[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < a.k) { slot[r] = a.inv[t * a.k + r]; wr[r] = a.w[t * a.k + r]; }
+      }
+      for (int sp = 0; sp < a.splits; ++sp) {
+#pragma unroll
+        for (int r = 0; r < KMAX; ++r) {
+          if (r < a.k) {
+            const float4 v = *reinterpret_cast<const float4*>(a.d + sp * rstride + (size_t)slot[r] * a.N + n);
+            d[r].x += v.x; d[r].y += v.y; d[r].z += v.z; d[r].w += v.w;
+          }
         }
-        acc[0] = __fadd_rn(acc[0], __fmul_rn(wr, d.x)); acc[1] = __fadd_rn(acc[1], __fmul_rn(wr, d.y));
-        acc[2] = __fadd_rn(acc[2], __fmul_rn(wr, d.z)); acc[3] = __fadd_rn(acc[3], __fmul_rn(wr, d.w));
+      }
+#pragma unroll
+      for (int r = 0; r < KMAX; ++r) {
+        if (r < a.k) {
+          acc[0] = __fadd_rn(acc[0], __fmul_rn(wr[r], d[r].x)); acc[1] = __fadd_rn(acc[1], __fmul_rn(wr[r], d[r].y));
+          acc[2] = __fadd_rn(acc[2], __fmul_rn(wr[r], d[r].z)); acc[3] = __fadd_rn(acc[3], __fmul_rn(wr[r], d[r].w));
+        }
       }
       for (int j = 0; j < 4; ++j) y[j] = round_bf16(acc[j]);
     }
@@ -162,9 +181,16 @@ cudaError_t launch_tail(const TailArgs& a, cudaStream_t s) {
   } else {
     if (a.N % 4 != 0) return cudaErrorInvalidValue;
     const size_t total4 = (size_t)a.M * a.N / 4;
-    int blocks = (int)((total4 + 255) / 256);
+    // Small row counts: 128-thread blocks over more SMs; else 256.
+    const int threads = total4 < (size_t)148 * 256 ? 128 : 256;
+    int blocks = (int)((total4 + threads - 1) / threads);
     if (blocks > 148 * 8) blocks = 148 * 8;
-    return launch_pdl(k_tail_elementwise, dim3(blocks), dim3(256), 0, s, a);
+    const int k = a.mode == TAIL_RESIDUAL ? 1 : a.k;
+    if (k <= 2) return launch_pdl(k_tail_elementwise<2>, dim3(blocks), dim3(threads), 0, s, a);
+    if (k <= 4) return launch_pdl(k_tail_elementwise<4>, dim3(blocks), dim3(threads), 0, s, a);
+    if (k <= 8) return launch_pdl(k_tail_elementwise<8>, dim3(blocks), dim3(threads), 0, s, a);
+    if (k <= 16) return launch_pdl(k_tail_elementwise<16>, dim3(blocks), dim3(threads), 0, s, a);
+    return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }
