@@ -8,7 +8,6 @@
 
 #include "../../include/moeffn.h"
 #include "common.cuh"
-#include "gemv.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_tma.cuh"
 #include "tmap.cuh"
@@ -53,8 +52,6 @@ int cuda_fail(cudaError_t e, const char* where) {
 
 constexpr int kSMs = 148;
 constexpr size_t kAlign = 256;
-constexpr size_t kStageBudget = 96 * 1024;      // shared memory per CTA for staged tokens
-constexpr size_t kStageMax = 200 * 1024;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -82,7 +79,8 @@ int check_qweight(const moeffn_qweight& w, const char* name, int rows, int cols)
   if (w.format == MOEFFN_Q_INT4_AFFINE_G32) {
     if (cols % 32 != 0) return fail(MOEFFN_ERR_INVALID, "%s: INT4-affine needs cols %% 32 == 0 (cols=%d)", name, cols);
     if (w.min == nullptr) return fail(MOEFFN_ERR_INVALID, "%s: INT4-affine needs a min array", name);
-    if ((reinterpret_cast<uintptr_t>(w.min) & 1u) != 0) return fail(MOEFFN_ERR_INVALID, "%s: min misaligned", name);
+    if (!aligned16(w.scale) || !aligned16(w.min))
+      return fail(MOEFFN_ERR_INVALID, "%s: INT4-affine scale and min must be 16-byte aligned", name);
   } else if (cols % 16 != 0) {
     return fail(MOEFFN_ERR_INVALID, "%s: INT8 needs cols %% 16 == 0 (cols=%d)", name, cols);
   }
@@ -104,19 +102,16 @@ int check_ffn(const moeffn_ffn& f, const char* name, int H, int I) {
 
 // ---- launch geometry -------------------------------------------------------
 
-int round_up8(int v) { return (v + 7) / 8 * 8; }
 
-// Rows per CTA so that about two CTAs per SM are launched.
-int rows_per_cta(int rows_total) {
-  int r = round_up8((rows_total + 2 * kSMs - 1) / (2 * kSMs));
-  return std::min(64, std::max(8, r));
-}
 
 // K split of a down projection: slices of at most 4096 (INT4), 3584 (Q4_K:
 // 14 blocks of 18 eight-byte elements) or 2048 (INT8) elements, a multiple of
 // 256 (16-byte aligned scale rows and TMA boxes of at most 256 eight-byte
-// elements); every split starts below K.
+// elements); every split starts below K. An INT4 matrix with K % 256 != 0
+// is not split: its scale rows (K / 16 bytes apart) could not be boxed, and
+// whole rows go through 1-D bulk copies.
 int down_slice(int K, int fmt) {
+  if (fmt == MOEFFN_Q_INT4_AFFINE_G32 && K % 256 != 0) return K;
   const int lim = fmt == MOEFFN_Q_INT8_ROW ? 2048 : fmt == MOEFFN_Q_Q4_K ? 3584 : 4096;
   const int s = (K + lim - 1) / lim;
   return ((K + s - 1) / s + 255) / 256 * 256;
@@ -136,17 +131,6 @@ int down_splits_any(int K) {
 constexpr size_t kTmaSmemBudget = 200 * 1024;
 constexpr size_t kTmaXBudget = 72 * 1024;
 
-// The bulk copies need 16-byte aligned sources, destinations and sizes. A
-// stage is 8 whole rows (rows per CTA are a multiple of 8, and every valid FFN
-// matrix has a multiple of 8 rows), so unsplit INT4 rows need only K % 32 ==
-// 0; a matrix split along K loads its scale and min boxes through 2-D tensor
-// maps, whose row stride (K / 16 bytes) must be a multiple of 16: K % 256 == 0.
-bool tma_ok(const moeffn_qweight& w) {
-  if (w.format == MOEFFN_Q_INT8_ROW || w.format == MOEFFN_Q_Q4_K) return true;
-  if (w.rows % 8 != 0 || !aligned16(w.scale) || !aligned16(w.min)) return false;
-  return w.cols % 256 == 0 || down_splits(w.cols, MOEFFN_Q_INT4_AFFINE_G32) == 1;
-}
-bool tma_ok(const moeffn_ffn& f) { return tma_ok(f.gate) && tma_ok(f.up) && tma_ok(f.down); }
 
 struct TmaGeom {
   int tokens, stages, mt;
@@ -170,13 +154,12 @@ TmaGeom tma_geom(int fmt, int nm, int klen, int want_tokens) {
   return g;
 }
 
-int stage_tokens(int fmt, int klen, int want) {
-  const size_t per = gemv_stage_bytes(fmt, klen, 1);
-  int t = (int)std::max<size_t>(1, kStageBudget / per);
-  return std::max(1, std::min(want, t));
+// Whether a dense FFN's weight stages fit the bulk-copy GEMV's ring (one
+// token row staged; more rows are staged in blocks that fit).
+bool gemv_fits(const moeffn_ffn& f, int H, int I) {
+  const int fmt = f.gate.format, dfmt = f.down.format;
+  return tma_geom(fmt, 2, H, 1).ok && tma_geom(dfmt, 1, down_slice(I, dfmt), 1).ok;
 }
-
-int mt_for(int tokens) { return tokens <= 1 ? 1 : 2; }
 
 // ---- tensor-core GEMM eligibility and geometry ------------------------------
 
@@ -390,7 +373,9 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
   *splits_out = splits;
   const TmaGeom gu = tma_geom(fmt, 2, H, M);
   const TmaGeom dn = tma_geom(dfmt, 1, ks, M);
-  if (tma_ok(f) && gu.ok && dn.ok) {
+  if (!gu.ok || !dn.ok)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "hidden size %d / intermediate size %d: the bulk-copy GEMV's stages do not fit", H, I);
+  {
     TmaGemvArgs g{};
     g.fmt = fmt;
     g.act = act;
@@ -462,49 +447,6 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     return MOEFFN_OK;
   }
 
-  // The register-load GEMV below takes the INT8 and INT4 block types only.
-  if (fmt == MOEFFN_Q_Q4_K || dfmt == MOEFFN_Q_Q4_K)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "Q4_K weights need the bulk-copy GEMV (shape or alignment not eligible)");
-  if (norm_w != nullptr) {
-    if ((rc = launch_prenorm(x, norm_w, eps, M, H, w, s)) != MOEFFN_OK) return rc;
-    x = w.m;
-  }
-  GateUpArgs g{};
-  g.fmt = fmt;
-  g.act = act;
-  g.K = H;
-  g.g = to_qw(f.gate);
-  g.u = to_qw(f.up);
-  g.N = I;
-  g.x = x;
-  g.M = M;
-  g.topk = 1;
-  g.routed_jobs = 1;
-  g.out = w.acts;
-  g.rows_per_cta = rows_per_cta(I);
-  g.stage_tokens = stage_tokens(fmt, H, M);
-  {
-    ProfScope ps("gateup_gemv", s);
-    MOEFFN_CHECK_CUDA(launch_gateup(g, (I + g.rows_per_cta - 1) / g.rows_per_cta, 1, mt_for(M), s), "gate/up launch");
-  }
-  DownArgs d{};
-  d.fmt = dfmt;
-  d.K = I;
-  d.N = H;
-  d.w = to_qw(f.down);
-  d.in = w.acts;
-  d.M = M;
-  d.slots = M;
-  d.d = w.d;
-  d.ks_len = ks;
-  d.rows_per_cta = rows_per_cta(H * splits);
-  d.stage_tokens = stage_tokens(dfmt, d.ks_len, M);
-  {
-    ProfScope ps("down_gemv", s);
-    MOEFFN_CHECK_CUDA(launch_down(d, (H + d.rows_per_cta - 1) / d.rows_per_cta, splits, 1, mt_for(M), s),
-                      "down launch");
-  }
-  return MOEFFN_OK;
 }
 
 }  // namespace
@@ -523,7 +465,6 @@ struct moeffn_moe_plan {
   const float* expert_scale = nullptr;         // per-expert routing scale (null: ones)
   const uint16_t* shared_post_norm = nullptr;  // Gemma form: the shared branch's post-FFN norm weight
   float shared_post_norm_eps = 0.f;
-  bool tma;               // every expert (and the shared one) fits the TMA GEMV
   QW* d_gate = nullptr;   // device tables [E]
   QW* d_up = nullptr;
   QW* d_down = nullptr;
@@ -603,8 +544,8 @@ int dense_entry(const char* who, const moeffn_ffn* w, const uint16_t* x, const u
   }
   if (!aligned16(x) || !aligned16(residual)) return fail(MOEFFN_ERR_INVALID, "%s: x/residual not 16-byte aligned", who);
   if (norm_w == nullptr && x == residual) return fail(MOEFFN_ERR_INVALID, "%s: x aliases residual", who);
-  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax || gemv_stage_bytes(w->down.format, down_slice(I, w->down.format), 1) > kStageMax)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: hidden size %d too large for the staged GEMV", who, H);
+  if (!gemv_fits(*w, H, I))
+    return fail(MOEFFN_ERR_UNSUPPORTED, "%s: hidden size %d too large for the bulk-copy GEMV's stages", who, H);
   Carve c{nullptr};
   carve_dense(c, M, H, I);
   if ((rc = check_ws(ws, ws_bytes, c.off)) != MOEFFN_OK) return rc;
@@ -659,8 +600,8 @@ int ffn_shared_expert(const moeffn_ffn* w, const uint16_t* x, const uint16_t* no
   if (rc != MOEFFN_OK) return rc;
   if (!aligned16(x) || !aligned16(h1_out)) return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: x/h1 not 16-byte aligned");
   if (x == h1_out) return fail(MOEFFN_ERR_INVALID, "ffn_shared_expert: x aliases h1_out");
-  if (gemv_stage_bytes(w->gate.format, H, 1) > kStageMax)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "ffn_shared_expert: hidden size %d too large", H);
+  if (!gemv_fits(*w, H, I))
+    return fail(MOEFFN_ERR_UNSUPPORTED, "ffn_shared_expert: hidden size %d too large for the bulk-copy GEMV's stages", H);
   Carve c{nullptr};
   carve_dense(c, M, H, I);
   if ((rc = check_ws(ws, ws_bytes, c.off)) != MOEFFN_OK) return rc;
@@ -794,16 +735,14 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   }
   if (desc->expert_scale != nullptr && (reinterpret_cast<uintptr_t>(desc->expert_scale) & 3u) != 0)
     return fail(MOEFFN_ERR_INVALID, "moe_plan_create: expert_scale not 4-byte aligned");
-  if (gemv_stage_bytes(MOEFFN_Q_INT4_AFFINE_G32, H, 1) > kStageMax)
-    return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: hidden size %d too large", H);
+  if (!tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, H, 1).ok ||
+      !tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 1, moe_split(Ie, Is).ks_len, 1).ok)
+    return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: hidden size %d too large for the bulk-copy GEMV's stages", H);
   auto* p = new moeffn_moe_plan();
   p->E = E; p->k = k; p->act = desc->act; p->H = H; p->Ie = Ie; p->Is = Is;
   p->router_fmt = desc->router.format;
   p->router = desc->router.q;
   p->has_shared = desc->shared != nullptr;
-  p->tma = true;
-  for (int e = 0; e < E; ++e) p->tma = p->tma && tma_ok(desc->experts[e]);
-  if (p->has_shared) p->tma = p->tma && tma_ok(*desc->shared);
   if (p->has_shared) {
     p->shared = *desc->shared;
     p->w_sg = desc->shared_gate != nullptr ? static_cast<const uint16_t*>(desc->shared_gate->q) : nullptr;
@@ -827,7 +766,7 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   }
   // Tensor maps for the down projections split along K (bulk-copy GEMV).
   const MoeSplit sp = moe_split(Ie, Is);
-  if (p->tma && (sp.routed > 1 || sp.shared > 1)) {
+  if (sp.routed > 1 || sp.shared > 1) {
     std::vector<QWMaps> maps(E);
     bool ok = true;
     for (int e = 0; e < E && ok; ++e)
@@ -1059,7 +998,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
       MOEFFN_CHECK_CUDA(launch_tc_gemm(d, row_tiles, std::max(tc_splits_r, tc_splits_s), jobs, s),
                         "phase-2 GEMM launch");
     }
-  } else if (p->tma && gu.ok && dn.ok) {
+  } else {
     TmaGemvArgs g{};
     g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
     g.act = p->act;
@@ -1127,65 +1066,6 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
       ProfScope ps("phase2_down_gemv_tma", s);
       MOEFFN_CHECK_CUDA(launch_tma_gemv(d, 1, dn.mt, splits, jobs, s), "phase-2 launch");
     }
-  } else {
-  GateUpArgs g{};
-  g.fmt = MOEFFN_Q_INT4_AFFINE_G32;
-  g.act = p->act;
-  g.K = H;
-  g.g_tab = p->d_gate;
-  g.u_tab = p->d_up;
-  g.N = Ie;
-  if (p->has_shared) {
-    g.sg = to_qw(p->shared.gate);
-    g.su = to_qw(p->shared.up);
-    g.Ns = Is;
-  }
-  g.x = x;
-  g.M = M;
-  g.topk = k;
-  g.perm = w.perm;
-  g.offsets = w.offsets;
-  g.union_list = w.union_list;
-  g.n_union = w.n_union;
-  g.routed_jobs = routed_jobs;
-  g.out = w.acts;
-  g.out_s = w.acts_s;
-  // Expected active rows: min(E, P) experts of Ie rows (+ the shared expert).
-  g.rows_per_cta = rows_per_cta(std::min(E, P) * Ie + Is);
-  g.stage_tokens = stage_tokens(g.fmt, H, max_tok);
-  const int gx = (std::max(Ie, Is) + g.rows_per_cta - 1) / g.rows_per_cta;
-  {
-    ProfScope ps("phase1_gateup_gemv", s);
-    MOEFFN_CHECK_CUDA(launch_gateup(g, gx, jobs, mt_for(std::min(M, 2)), s), "phase-1 launch");
-  }
-
-  DownArgs d{};
-  d.fmt = MOEFFN_Q_INT4_AFFINE_G32;
-  d.K = Ie;
-  d.N = H;
-  d.tab = p->d_down;
-  if (p->has_shared) d.ws = to_qw(p->shared.down);
-  d.Ks = Is;
-  d.in = w.acts;
-  d.in_s = w.acts_s;
-  d.M = M;
-  d.slots = P;
-  d.offsets = w.offsets;
-  d.union_list = w.union_list;
-  d.n_union = w.n_union;
-  d.routed_jobs = routed_jobs;
-  d.d = w.d;
-  d.d_s = w.d_s;
-  // One slice length for routed and shared jobs; each job has its own count.
-  d.ks_len = sp.ks_len;
-  d.rows_per_cta = rows_per_cta(H * std::max(1, std::min(E, P) / 4));
-  d.stage_tokens = stage_tokens(d.fmt, d.ks_len, max_tok);
-  {
-    ProfScope ps("phase2_down_gemv", s);
-    MOEFFN_CHECK_CUDA(launch_down(d, (H + d.rows_per_cta - 1) / d.rows_per_cta, std::max(splits_r, splits_sh), jobs,
-                                  mt_for(std::min(M, 2)), s),
-                      "phase-2 launch");
-  }
   }
 
   TailArgs t{};

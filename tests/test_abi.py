@@ -86,6 +86,12 @@ def test_refusals_before_launch():
     mixed.up = _fake_qweight(lib, lib.Q_INT8_ROW, 512, 256, 0x30000000)
     assert L.ffn_dense(ctypes.byref(mixed), x, r, 2, 0, ws, 1 << 30, None) == -2
     assert b"gate and up" in L.moeffn_last_error()
+    unal = _fake_ffn(lib, lib.Q_INT4_AFFINE_G32, 256, 512)
+    unal.down = lib._QWeight(lib.Q_INT4_AFFINE_G32, 256, 512, 0x30000000, 0x30100002, 0x30200000)   # scale + 2 bytes
+    assert L.ffn_dense(ctypes.byref(unal), x, r, 2, 0, ws, 1 << 30, None) == -1
+    assert b"16-byte" in L.moeffn_last_error()
+    huge = _fake_ffn(lib, lib.Q_INT8_ROW, 65536, 512)                                 # stages do not fit
+    assert L.ffn_dense(ctypes.byref(huge), x, r, 2, 0, ws, 1 << 40, None) == -2
     q4k = _fake_ffn(lib, lib.Q_Q4_K, 256 + 128, 512)                                 # Q4_K: K % 256 != 0
     assert L.ffn_dense(ctypes.byref(q4k), x, r, 2, 0, ws, 1 << 30, None) == -1
     assert b"256" in L.moeffn_last_error()

@@ -108,7 +108,7 @@ DENSE_SMALL = [
     (2, dict(H=640, I=1056), FMT_INT4_G32),     # K % 256 != 0, unsplit: bulk-copy GEMV
     (2, dict(H=512, I=1280), FMT_INT4_G32),     # bulk-copy GEMV, ragged CTA row ranges
     (2, dict(H=256, I=4352), FMT_INT4_G32),     # down split along K: 2-D tensor-map boxes
-    (2, dict(H=256, I=4384), FMT_INT4_G32),     # split K with K % 256 != 0: register-load GEMV
+    (2, dict(H=256, I=4384), FMT_INT4_G32),     # K % 256 != 0 and K > 4096: the down projection is not split
 ]
 
 
@@ -198,7 +198,7 @@ def test_shared_expert_small(M, shape):
 
 
 MOE_SMALL = [
-    dict(cfg=4, H=256, I=96, E=16, k=4, I_s=64),     # register-load GEMV path
+    dict(cfg=4, H=256, I=96, E=16, k=4, I_s=64),     # expert width 96: unsplit down rows, K % 256 != 0
     dict(cfg=5, H=320, I=192, E=8, k=2, I_s=0),
     dict(cfg=4, H=256, I=64, E=4, k=4, I_s=128),
     dict(cfg=4, H=512, I=256, E=16, k=4, I_s=256),   # bulk-copy GEMV path
@@ -233,7 +233,7 @@ def _norm_w(H, seed):
 PRENORM_DENSE = [
     (2, dict(H=512, I=1024)),      # INT4: GEMV staging folds the norm (M <= 5), a norm launch before the GEMMs
     (1, dict(H=256, I=416)),       # INT8
-    (2, dict(H=640, I=1056)),      # K % 256 != 0: register-load GEMV after a norm launch
+    (2, dict(H=640, I=1056)),      # K % 256 != 0: unsplit rows; tensor-core path refused, a norm launch before the GEMV
 ]
 
 
