@@ -1,6 +1,7 @@
 // C ABI of libmoeffn.so: argument validation, workspace carving and the
 // launch sequence of each layer kind. See include/moeffn.h for the contract.
 #include <algorithm>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <string>
@@ -926,10 +927,13 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     }
     // One CTA should cover a whole expert's token rows, since a second token
     // tile dequantizes every weight of the expert again: the token tile is
-    // sized for the mean load per expert plus half again for the routing
-    // spread (an expert holds at most M rows).
+    // sized for the mean load per expert plus the larger of a quarter of it
+    // and 2.5 standard deviations of the routing spread (about sqrt(mean)); an
+    // expert holds at most M rows. Keeping the tile narrow leaves TMEM for a
+    // deeper A stage ring (a tile of 160 columns leaves three stages, 192 two).
     const int per_expert = std::max(1, P / std::min(E, P));
-    const int ntile = std::min(kTcMaxTok, (std::min(M, per_expert + per_expert / 2 + 1) + 15) & ~15);
+    const int spread = std::max(per_expert / 4, (int)(2.5 * std::sqrt((double)per_expert)) + 1);
+    const int ntile = std::min(kTcMaxTok, (std::min(M, per_expert + spread) + 15) & ~15);
     const int tt = (M + ntile - 1) / ntile;
     TcGemmArgs g{};
     g.fmt = MOEFFN_Q_INT4_AFFINE_G32;

@@ -38,7 +38,7 @@
 //
 // TMEM columns: accumulator of A tile t at [t * ntile, (t + 1) * ntile); a ring
 // of A stages (two K groups each: 32 columns per A tile) after them; the
-// ring depth SA (at most 6) is what the accumulators leave. Waits
+// ring depth SA (2 to 7) is what the accumulators leave. Waits
 // suspend the waiting thread (mbarrier.try_wait) rather than spin, so the
 // producer and MMA threads take no issue slots from the dequantizing warps.
 // Modes: GATEUP writes bf16(act(gate) * up); DOWN writes fp32 partial sums
@@ -271,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   const int nW = klen / F::kKTile;                  // weight stages
   const int tn = min(ntile, job.ntok - t0);         // valid token rows
   const int nmma = (tn + 15) & ~15;                 // MMA N
-  const int SA = min(8, (kTmemCols - kTilesA * ntile) / kAStageCols) & ~1;   // A ring depth (even)
+  const int SA = min(8, (kTmemCols - kTilesA * ntile) / kAStageCols);   // A ring depth (2..7)
   const uint32_t a_col0 = (uint32_t)(kTilesA * ntile);
 
   // ---- shared memory carve (1024-byte aligned operand tiles) -------------
