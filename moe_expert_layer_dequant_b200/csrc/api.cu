@@ -159,7 +159,7 @@ TmaGeom tma_geom(int fmt, int nm, int klen, int want_tokens) {
 // token row staged; more rows are staged in blocks that fit).
 bool gemv_fits(const moeffn_ffn& f, int H, int I) {
   const int fmt = f.gate.format, dfmt = f.down.format;
-  return tma_geom(fmt, 2, H, 1).ok && tma_geom(dfmt, 1, down_slice(I, dfmt), 1).ok;
+  return tma_geom(fmt, 2, H, 1).ok && tma_geom(dfmt, 2, down_slice(I, dfmt), 1).ok;   // down: row pairs
 }
 
 // ---- tensor-core GEMM eligibility and geometry ------------------------------
@@ -373,7 +373,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
   const int ks = down_slice(I, dfmt), splits = down_splits(I, dfmt);
   *splits_out = splits;
   const TmaGeom gu = tma_geom(fmt, 2, H, M);
-  const TmaGeom dn = tma_geom(dfmt, 1, ks, M);
+  const TmaGeom dn = tma_geom(dfmt, 2, ks, M);   // row pairs: the two-matrix stage
   if (!gu.ok || !dn.ok)
     return fail(MOEFFN_ERR_UNSUPPORTED, "hidden size %d / intermediate size %d: the bulk-copy GEMV's stages do not fit", H, I);
   {
@@ -436,6 +436,7 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.ctas_per_job = std::max(1, kSMs / splits);
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;
+    d.row_pairs = 1;
     if (res != nullptr) {
       d.tile_cnt = w.cnt;
       d.res = res;
@@ -737,7 +738,7 @@ int moe_plan_create(const moeffn_moe_desc* desc, moeffn_moe_plan** plan) {
   if (desc->expert_scale != nullptr && (reinterpret_cast<uintptr_t>(desc->expert_scale) & 3u) != 0)
     return fail(MOEFFN_ERR_INVALID, "moe_plan_create: expert_scale not 4-byte aligned");
   if (!tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, H, 1).ok ||
-      !tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 1, moe_split(Ie, Is).ks_len, 1).ok)
+      !tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, moe_split(Ie, Is).ks_len, 1).ok)
     return fail(MOEFFN_ERR_UNSUPPORTED, "moe_plan_create: hidden size %d too large for the bulk-copy GEMV's stages", H);
   auto* p = new moeffn_moe_plan();
   p->E = E; p->k = k; p->act = desc->act; p->H = H; p->Ie = Ie; p->Is = Is;
@@ -915,7 +916,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
   const int splits_r = sp.routed, splits_sh = sp.shared;
   const int splits = std::max(splits_r, splits_sh);
   const TmaGeom gu = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, H, max_tok);
-  const TmaGeom dn = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 1, sp.ks_len, max_tok);
+  const TmaGeom dn = tma_geom(MOEFFN_Q_INT4_AFFINE_G32, 2, sp.ks_len, max_tok);   // row pairs
   int tc_splits_r = splits_r, tc_splits_s = splits_sh;
   const bool use_tc = p->tc && M >= kTcMinMoeTokens && aligned16(x);
   if (use_tc) {
@@ -1061,6 +1062,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     d.out_d_s = w.d_s;
     d.ks_len = sp.ks_len;
     d.use_maps = splits > 1;
+    d.row_pairs = 1;
     d.maps = p->d_maps;
     d.maps_s = p->d_maps_s;
     d.ctas_per_job = std::max(1, kSMs / (jobs * splits));

@@ -65,8 +65,14 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 // depth S is a multiple of G, so every slot is waited on by one group only,
 // in stage order: a waiter is never two phases ahead of a slot's barriers
 // (whose phase parity would then alias the previous use).
-template <int FMT, int MT, int NM, int NC, int G>
+//
+// PR (row pairs, a single matrix: the down projection): a stage holds 2R
+// consecutive rows of one matrix, as NM = 2 holds R rows of two, and each
+// warp computes rows n and n + R, so that the activations it loads from shared
+// memory serve two rows.
+template <int FMT, int MT, int NM, int NC, int G, bool PR = false>
 __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_constant__ TmaGemvArgs a) {
+  static_assert(!PR || NM == 2, "row pairs use the two-matrix stage layout");
   using C = Codes<FMT>;
   constexpr bool kInt4 = (FMT == FMT_INT4_G32);
   constexpr bool kQ4K = (FMT == FMT_Q4K);
@@ -89,7 +95,8 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   const int k0 = blockIdx.y * a.ks_len;
   if (k0 >= job.K) return;
   const int klen = min(a.ks_len, job.K - k0);
-  const int rpc = ((job.N + a.ctas_per_job - 1) / a.ctas_per_job + R - 1) / R * R;
+  constexpr int RS = PR ? 2 * R : R;   // rows per stage
+  const int rpc = ((job.N + a.ctas_per_job - 1) / a.ctas_per_job + RS - 1) / RS * RS;
   const int r0 = blockIdx.x * rpc;
   const int r1 = min(job.N, r0 + rpc);
   if (r0 >= r1) return;
@@ -130,7 +137,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   }
   __syncthreads();
 
-  const int row_stages = (r1 - r0 + R - 1) / R;
+  const int row_stages = (r1 - r0 + RS - 1) / RS;
   const int tok_blocks = (job.ntok + a.stage_tokens - 1) / a.stage_tokens;
   const int total = row_stages * tok_blocks;
   const int row_bytes = kInt4 ? job.K / 2 : kQ4K ? job.K / Q4K::kBlock * Q4K::kBytes : job.K;
@@ -147,7 +154,7 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
         const int slot = s % S, use = s / S;
         if (a.inject_stop > 0 && s >= a.inject_stop - 1) break;   // injected producer failure (tests)
         if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, wait_ns)) break;
-        const int n0 = r0 + (s % row_stages) * R;
+        const int n0 = r0 + (s % row_stages) * RS;
         const int nr = min(R, r1 - n0);
         uint8_t* st = stage0 + (size_t)slot * stage_bytes;
         uint8_t* dsc = st + (size_t)NM * R * cs;
@@ -158,25 +165,32 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
 #pragma unroll
           for (int i = 0; i < NM; ++i) {
             // x in 8-byte elements: 16 INT4 codes, 8 INT8 codes, or 18 per Q4_K block
-            tma_load_2d(st + (size_t)i * R * cs, &jm[i].codes, kInt4 ? k0 / 16 : kQ4K ? k0 / Q4K::kBlock * 18 : k0 / 8,
-                        n0, &full[slot]);
+            const QWMaps& mp = jm[PR ? 0 : i];
+            const int ny = n0 + (PR ? i * R : 0);   // rows past the end arrive as zeros
+            tma_load_2d(st + (size_t)i * R * cs, &mp.codes, kInt4 ? k0 / 16 : kQ4K ? k0 / Q4K::kBlock * 18 : k0 / 8,
+                        ny, &full[slot]);
             if (kInt4) {
-              tma_load_2d(dsc + (size_t)i * R * gst * 2, &jm[i].scale, k0 / 32, n0, &full[slot]);
-              tma_load_2d(dmn + (size_t)i * R * gst * 2, &jm[i].mn, k0 / 32, n0, &full[slot]);
+              tma_load_2d(dsc + (size_t)i * R * gst * 2, &mp.scale, k0 / 32, ny, &full[slot]);
+              tma_load_2d(dmn + (size_t)i * R * gst * 2, &mp.mn, k0 / 32, ny, &full[slot]);
             }
           }
         } else {
           // Whole rows are contiguous: one copy per array for the stage.
-          mbar_arrive_expect_tx(&full[slot], (uint32_t)(NM * nr * (cs + 4 * gst)));
+          const int nr1 = PR ? max(0, min(R, r1 - (n0 + R))) : nr;   // rows of the second half
+          mbar_arrive_expect_tx(&full[slot], (uint32_t)((nr + (NM == 2 ? nr1 : 0)) * (cs + 4 * gst)));
 #pragma unroll
           for (int i = 0; i < NM; ++i) {
-            bulk_g2s(st + (size_t)i * R * cs, job.m[i].q + (size_t)n0 * row_bytes, (uint32_t)(nr * cs), &full[slot]);
-            if (kInt4) {
-              const size_t go = (size_t)n0 * row_groups * 2;
-              bulk_g2s(dsc + (size_t)i * R * gst * 2, reinterpret_cast<const uint8_t*>(job.m[i].scale) + go,
-                       (uint32_t)(nr * gst * 2), &full[slot]);
-              bulk_g2s(dmn + (size_t)i * R * gst * 2, reinterpret_cast<const uint8_t*>(job.m[i].mn) + go,
-                       (uint32_t)(nr * gst * 2), &full[slot]);
+            const QW& mq = job.m[PR ? 0 : i];
+            const int ni = n0 + (PR ? i * R : 0), cnt = i == 0 ? nr : nr1;
+            if (cnt > 0) {
+              bulk_g2s(st + (size_t)i * R * cs, mq.q + (size_t)ni * row_bytes, (uint32_t)(cnt * cs), &full[slot]);
+              if (kInt4) {
+                const size_t go = (size_t)ni * row_groups * 2;
+                bulk_g2s(dsc + (size_t)i * R * gst * 2, reinterpret_cast<const uint8_t*>(mq.scale) + go,
+                         (uint32_t)(cnt * gst * 2), &full[slot]);
+                bulk_g2s(dmn + (size_t)i * R * gst * 2, reinterpret_cast<const uint8_t*>(mq.mn) + go,
+                         (uint32_t)(cnt * gst * 2), &full[slot]);
+              }
             }
           }
         }
@@ -239,11 +253,14 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
     for (int rs = grp; rs < row_stages; rs += G) {
       const int s = tbi * row_stages + rs;
       const int slot = s % S, use = s / S;
-      const int n = r0 + rs * R + wr;
+      const int n = r0 + rs * RS + wr;
       float row_scale[NM];
       if (FMT == FMT_INT8_ROW && n < r1) {
 #pragma unroll
-        for (int i = 0; i < NM; ++i) row_scale[i] = __half2float(__ldg(job.m[i].scale + n));
+        for (int i = 0; i < NM; ++i) {
+          const int ni = n + (PR ? i * R : 0);
+          row_scale[i] = ni < r1 ? __half2float(__ldg(job.m[PR ? 0 : i].scale + ni)) : 0.f;
+        }
       }
       // After a timed-out wait (a fault already recorded) the warp stops
       // computing but still takes part in every barrier below.
@@ -389,13 +406,17 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
             const int tok = tb + tc + t;
             if (lane == 0 && tok < tn + tb) {
               const int slot_out = job.slot0 + tok;
-              if (NM == 2) {
+              if (NM == 2 && !PR) {
                 uint16_t* out = job.shared ? a.out_act_s : a.out_act;
                 out[(size_t)slot_out * job.N + n] = float_to_bf16_bits(gated_act(v[0], v[NM - 1], a.act));
               } else {
                 float* d = job.shared ? a.out_d_s : a.out_d;
                 const int nslots = job.shared ? a.M : a.slots;
-                d[((size_t)blockIdx.y * nslots + slot_out) * job.N + n] = v[0];
+#pragma unroll
+                for (int i = 0; i < NM; ++i) {
+                  const int ni = n + (PR ? i * R : 0);
+                  if (i == 0 || ni < r1) d[((size_t)blockIdx.y * nslots + slot_out) * job.N + ni] = v[i];
+                }
               }
             }
           }
@@ -450,6 +471,17 @@ cudaError_t launch_fmt(const TmaGemvArgs& a, int mt, dim3 grid, size_t smem, cud
   return mt == 1 ? launch_one<FMT, 1, NM>(a, grid, smem, s) : launch_one<FMT, 2, NM>(a, grid, smem, s);
 }
 
+// Row pairs of one matrix: the two-matrix stage layout and consumer groups.
+template <int FMT, int MT>
+cudaError_t launch_pairs(const TmaGemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+  constexpr int G = tma_groups(FMT, 2);
+  auto kern = k_gemv_tma<FMT, MT, 2, kTmaConsumers, G, true>;
+  static bool opted[64] = {};
+  const cudaError_t e = opt_in_smem(kern, 227 * 1024, opted);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * G + 1)), smem, s, a);
+}
+
 }  // namespace
 
 size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
@@ -474,8 +506,14 @@ size_t tma_gemv_stage_bytes(int fmt, int nm, int klen) {
 }
 
 cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, int jobs, cudaStream_t s) {
-  const size_t smem = tma_gemv_smem(a.fmt, nm, a.ks_len, a.stage_tokens, mt, a.stages);
   const dim3 grid(a.ctas_per_job, splits, jobs);
+  if (nm == 1 && a.row_pairs) {
+    const size_t smem = tma_gemv_smem(a.fmt, 2, a.ks_len, a.stage_tokens, mt, a.stages);
+    if (a.fmt == FMT_INT4_G32) return mt == 1 ? launch_pairs<FMT_INT4_G32, 1>(a, grid, smem, s) : launch_pairs<FMT_INT4_G32, 2>(a, grid, smem, s);
+    if (a.fmt == FMT_Q4K) return mt == 1 ? launch_pairs<FMT_Q4K, 1>(a, grid, smem, s) : launch_pairs<FMT_Q4K, 2>(a, grid, smem, s);
+    return mt == 1 ? launch_pairs<FMT_INT8_ROW, 1>(a, grid, smem, s) : launch_pairs<FMT_INT8_ROW, 2>(a, grid, smem, s);
+  }
+  const size_t smem = tma_gemv_smem(a.fmt, nm, a.ks_len, a.stage_tokens, mt, a.stages);
   if (a.fmt == FMT_INT4_G32)
     return nm == 2 ? launch_fmt<FMT_INT4_G32, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_INT4_G32, 1>(a, mt, grid, smem, s);
   if (a.fmt == FMT_Q4K)

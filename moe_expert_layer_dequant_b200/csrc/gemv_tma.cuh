@@ -61,6 +61,8 @@ struct TmaGemvArgs {
   const uint16_t* norm_w;      // dense gate/up, unsplit K: normalize x on staging (RMSNorm weight [K]), or null
   float eps;
   int ks_len;                  // K elements per split (INT4, Q4_K: multiple of 256)
+  int row_pairs;               // single-matrix (down) launch: stages of 2 x 8 rows, two rows per warp;
+                               // stages and stage_tokens from the two-matrix geometry
   int ctas_per_job;
   int stage_tokens;
   int stages;
