@@ -148,7 +148,7 @@ TmaGeom tma_geom(int fmt, int nm, int klen, int want_tokens) {
   const size_t st = tma_gemv_stage_bytes(fmt, nm, klen);
   int stages = base + 2 * st <= kTmaSmemBudget ? (int)std::min<size_t>(8, (kTmaSmemBudget - base) / st) : 0;
   // Each ring slot must belong to one consumer group (see gemv_tma.cu).
-  const int groups = tma_groups(fmt, nm);
+  const int groups = kTmaGroups;
   stages -= stages % groups;
   g.stages = stages;
   g.ok = stages >= groups && stages >= 2;
@@ -436,7 +436,6 @@ int run_dense_ffn(const moeffn_ffn& f, const uint16_t* x, int M, int H, int I, i
     d.ctas_per_job = std::max(1, kSMs / splits);
     d.stage_tokens = dn.tokens;
     d.stages = dn.stages;
-    d.row_pairs = 1;
     if (res != nullptr) {
       d.tile_cnt = w.cnt;
       d.res = res;
@@ -1062,7 +1061,6 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     d.out_d_s = w.d_s;
     d.ks_len = sp.ks_len;
     d.use_maps = splits > 1;
-    d.row_pairs = 1;
     d.maps = p->d_maps;
     d.maps_s = p->d_maps_s;
     d.ctas_per_job = std::max(1, kSMs / (jobs * splits));

@@ -66,10 +66,10 @@ __device__ __forceinline__ void consumer_sync(int nthreads) {
 // in stage order: a waiter is never two phases ahead of a slot's barriers
 // (whose phase parity would then alias the previous use).
 //
-// PR (row pairs, a single matrix: the down projection): a stage holds 2R
-// consecutive rows of one matrix, as NM = 2 holds R rows of two, and each
-// warp computes rows n and n + R, so that the activations it loads from shared
-// memory serve two rows.
+// NM = 2: gate and up, R rows of each per stage. PR (row pairs, a single
+// matrix: the down projection): a stage holds 2R consecutive rows of one
+// matrix in the same layout, and each warp computes rows n and n + R, so that
+// the activations it loads from shared memory serve two rows.
 template <int FMT, int MT, int NM, int NC, int G, bool PR = false>
 __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_constant__ TmaGemvArgs a) {
   static_assert(!PR || NM == 2, "row pairs use the two-matrix stage layout");
@@ -456,30 +456,26 @@ __global__ void __launch_bounds__(32 * (NC * G + 1), 1) k_gemv_tma(const __grid_
   }
 }
 
-template <int FMT, int MT, int NM>
+// PR: one matrix in row pairs (the two-matrix stage layout); else gate + up.
+template <int FMT, int MT, bool PR>
 cudaError_t launch_one(const TmaGemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-  constexpr int G = tma_groups(FMT, NM);
-  auto kern = k_gemv_tma<FMT, MT, NM, kTmaConsumers, G>;
+  auto kern = k_gemv_tma<FMT, MT, 2, kTmaConsumers, kTmaGroups, PR>;
   static bool opted[64] = {};   // opted in to the 227 KB maximum
   const cudaError_t e = opt_in_smem(kern, 227 * 1024, opted);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * G + 1)), smem, s, a);
+  return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * kTmaGroups + 1)), smem, s, a);
 }
 
-template <int FMT, int NM>
+template <int FMT, bool PR>
 cudaError_t launch_fmt(const TmaGemvArgs& a, int mt, dim3 grid, size_t smem, cudaStream_t s) {
-  return mt == 1 ? launch_one<FMT, 1, NM>(a, grid, smem, s) : launch_one<FMT, 2, NM>(a, grid, smem, s);
+  return mt == 1 ? launch_one<FMT, 1, PR>(a, grid, smem, s) : launch_one<FMT, 2, PR>(a, grid, smem, s);
 }
 
-// Row pairs of one matrix: the two-matrix stage layout and consumer groups.
-template <int FMT, int MT>
-cudaError_t launch_pairs(const TmaGemvArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
-  constexpr int G = tma_groups(FMT, 2);
-  auto kern = k_gemv_tma<FMT, MT, 2, kTmaConsumers, G, true>;
-  static bool opted[64] = {};
-  const cudaError_t e = opt_in_smem(kern, 227 * 1024, opted);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(kern, grid, dim3(32 * (kTmaConsumers * G + 1)), smem, s, a);
+template <bool PR>
+cudaError_t launch_any(const TmaGemvArgs& a, int mt, dim3 grid, size_t smem, cudaStream_t s) {
+  if (a.fmt == FMT_INT4_G32) return launch_fmt<FMT_INT4_G32, PR>(a, mt, grid, smem, s);
+  if (a.fmt == FMT_Q4K) return launch_fmt<FMT_Q4K, PR>(a, mt, grid, smem, s);
+  return launch_fmt<FMT_INT8_ROW, PR>(a, mt, grid, smem, s);
 }
 
 }  // namespace
@@ -488,7 +484,7 @@ size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
 
 size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages) {
   const bool affine = fmt == FMT_INT4_G32 || fmt == FMT_Q4K;   // staged chunk sums
-  const size_t red = gemv_norm_bytes(kTmaConsumers * tma_groups(fmt, nm));
+  const size_t red = gemv_norm_bytes(kTmaConsumers * kTmaGroups);
   const int nch = klen / (fmt == FMT_INT8_ROW ? 16 : 32);
   const int cbytes = fmt == FMT_INT8_ROW ? Codes<FMT_INT8_ROW>::kStageBytes : Codes<FMT_INT4_G32>::kStageBytes;
   const int tok_rows = (stage_tokens + mt - 1) / mt * mt;
@@ -507,18 +503,8 @@ size_t tma_gemv_stage_bytes(int fmt, int nm, int klen) {
 
 cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, int jobs, cudaStream_t s) {
   const dim3 grid(a.ctas_per_job, splits, jobs);
-  if (nm == 1 && a.row_pairs) {
-    const size_t smem = tma_gemv_smem(a.fmt, 2, a.ks_len, a.stage_tokens, mt, a.stages);
-    if (a.fmt == FMT_INT4_G32) return mt == 1 ? launch_pairs<FMT_INT4_G32, 1>(a, grid, smem, s) : launch_pairs<FMT_INT4_G32, 2>(a, grid, smem, s);
-    if (a.fmt == FMT_Q4K) return mt == 1 ? launch_pairs<FMT_Q4K, 1>(a, grid, smem, s) : launch_pairs<FMT_Q4K, 2>(a, grid, smem, s);
-    return mt == 1 ? launch_pairs<FMT_INT8_ROW, 1>(a, grid, smem, s) : launch_pairs<FMT_INT8_ROW, 2>(a, grid, smem, s);
-  }
-  const size_t smem = tma_gemv_smem(a.fmt, nm, a.ks_len, a.stage_tokens, mt, a.stages);
-  if (a.fmt == FMT_INT4_G32)
-    return nm == 2 ? launch_fmt<FMT_INT4_G32, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_INT4_G32, 1>(a, mt, grid, smem, s);
-  if (a.fmt == FMT_Q4K)
-    return nm == 2 ? launch_fmt<FMT_Q4K, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_Q4K, 1>(a, mt, grid, smem, s);
-  return nm == 2 ? launch_fmt<FMT_INT8_ROW, 2>(a, mt, grid, smem, s) : launch_fmt<FMT_INT8_ROW, 1>(a, mt, grid, smem, s);
+  const size_t smem = tma_gemv_smem(a.fmt, 2, a.ks_len, a.stage_tokens, mt, a.stages);
+  return nm == 1 ? launch_any<true>(a, mt, grid, smem, s) : launch_any<false>(a, mt, grid, smem, s);
 }
 
 cudaError_t encode_qw_maps(QWMaps* m, int fmt, const QW& w, int N, int K, int ks_len) {

@@ -7,11 +7,11 @@
 namespace moeffn {
 
 constexpr int kTmaConsumers = 8;  // consumer warps per group = rows per stage
-// Consumer groups, taking stages in turn: three for a single INT4 or Q4_K
-// matrix (the down projection; more warps to hide the per-stage arithmetic latency), two
-// otherwise (the fused gate/up pair's larger stages leave room for fewer slots,
-// and the INT8 consumers need more registers than 800 threads allow).
-constexpr int tma_groups(int fmt, int nm) { return (nm == 1 && (fmt == FMT_INT4_G32 || fmt == FMT_Q4K)) ? 3 : 2; }
+// Consumer groups, taking stages in turn. Two: a stage of two matrices (gate
+// and up) or of one matrix's row pairs (down) is twice the bytes of a single
+// row set, and a third group (800 threads) would leave each thread too few
+// registers for the two rows' accumulators.
+constexpr int kTmaGroups = 2;
 // Token rows whose input norm the GEMV's staging applies (more: a norm launch first).
 constexpr int kGemvNormTokens = 8;
 // Shared memory of the staging's input-norm pass: inverse RMS per staged token
@@ -61,8 +61,6 @@ struct TmaGemvArgs {
   const uint16_t* norm_w;      // dense gate/up, unsplit K: normalize x on staging (RMSNorm weight [K]), or null
   float eps;
   int ks_len;                  // K elements per split (INT4, Q4_K: multiple of 256)
-  int row_pairs;               // single-matrix (down) launch: stages of 2 x 8 rows, two rows per warp;
-                               // stages and stage_tokens from the two-matrix geometry
   int ctas_per_job;
   int stage_tokens;
   int stages;
@@ -75,6 +73,9 @@ struct TmaGemvArgs {
 
 // Encodes the three maps of W[N][K] for boxes of [rows_per_stage][ks_len].
 cudaError_t encode_qw_maps(QWMaps* m, int fmt, const QW& w, int N, int K, int ks_len);
+// nm: 2 for the fused gate/up launch, 1 for a single matrix (the down
+// projection), whose stages hold row pairs: 2 x 8 rows, the bytes of a
+// two-matrix stage, so its geometry is that of nm = 2.
 size_t tma_gemv_smem(int fmt, int nm, int klen, int stage_tokens, int mt, int stages);
 size_t tma_gemv_stage_bytes(int fmt, int nm, int klen);
 cudaError_t launch_tma_gemv(const TmaGemvArgs& a, int nm, int mt, int splits, int jobs, cudaStream_t s);
