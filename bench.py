@@ -402,9 +402,18 @@ def run_ours(args, rank, world, local_rank):
         # bound: the larger of the weight-stream time and the tensor-core time
         tensor_bound = bool(dom_flops and "gemm_tc" in dom_name and bf16_tf > 0 and
                             dom_flops / (bf16_tf * 1e12) > dom_bytes / (hbm * 1e9))
+        # A GEMM timed inside seconds of back-to-back steps runs under the
+        # power cap: its denominator is the sustained bf16 figure (a GEMM loop
+        # of seconds); the burst figure (a kernel timed alone) is given too.
+        long_loop = sum(rep_ms) >= 1000.0 and bf16_sus > 0
         if tensor_bound:
             achieved = dom_flops / dom_avg_s / 1e12
-            roof_peak, roof_unit, roof_src = bf16_tf, "TFLOP/s", f"{peak_src} bf16 dense GEMM (burst)"
+            if long_loop:
+                roof_peak, roof_unit = bf16_sus, "TFLOP/s"
+                roof_src = (f"{peak_src} bf16 dense GEMM, sustained (the kernel runs inside {sum(rep_ms) / 1e3:.1f} s "
+                            f"of back-to-back steps under the power cap)")
+            else:
+                roof_peak, roof_unit, roof_src = bf16_tf, "TFLOP/s", f"{peak_src} bf16 dense GEMM (burst)"
         else:
             achieved = dom_bytes / dom_avg_s / 1e9 if dom_bytes else None
             roof_peak, roof_unit, roof_src = hbm, "GB/s", f"{peak_src} HBM copy bandwidth"
@@ -443,7 +452,9 @@ def run_ours(args, rank, world, local_rank):
                 "kernel": dom_name, "bound": "tensor" if tensor_bound else "hbm",
                 "achieved": round(achieved, 1) if achieved else None,
                 "peak": roof_peak, "peak_source": roof_src, "unit": roof_unit,
-                "frac": round(achieved / roof_peak, 4) if achieved else None, "traffic": traffic,
+                "frac": round(achieved / roof_peak, 4) if achieved else None,
+                "frac_of_burst_peak": (round(achieved / bf16_tf, 4) if tensor_bound and achieved and bf16_tf > 0 else None),
+                "traffic": traffic,
                 "algorithmic_bytes_per_launch": dom_bytes, "algorithmic_flops_per_launch": dom_flops,
                 "avg_launch_us": round(dom_avg_s * 1e6, 3),
                 "timing_note": "per-launch CUDA events on the launching stream; with programmatic dependent "

@@ -117,7 +117,7 @@ struct Job {
 __device__ __forceinline__ Job decode_job(const TcGemmArgs& a) {
   Job j{};
   j.valid = true;
-  const int z = blockIdx.z;
+  const int z = blockIdx.y;
   if (a.offsets == nullptr) {
     j.m0 = &a.w0; j.m1 = &a.w1; j.xmap = &a.xmap; j.rs0 = a.rscale0; j.rs1 = a.rscale1;
     j.N = a.N; j.K = a.K; j.ntok = a.M;
@@ -255,7 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_qgemm_tc(const __grid_constant_
   const Job job = decode_job(a);
   if (!job.valid) return;
   const int ntile = a.ntile;
-  const int tt = blockIdx.y % a.token_tiles, split = blockIdx.y / a.token_tiles;
+  // grid.z runs over token tiles (slowest) and K splits: every job's first
+  // token tile is scheduled before any later one, so the tiles past an
+  // expert's token count (which exit at once) come last, in the wave tail.
+  const int splits = (int)gridDim.z / a.token_tiles;
+  const int tt = blockIdx.z / splits, split = blockIdx.z % splits;
   const int t0 = tt * ntile;
   if (t0 >= job.ntok) return;
   // Weight rows of the CTA: GATEUP features f0..f0+127 of gate (tile 0) and
@@ -523,7 +527,7 @@ cudaError_t encode_tc_x_map(CUtensorMap* m, const uint16_t* x, int rows, int K, 
 cudaError_t launch_tc_gemm(const TcGemmArgs& a, int row_tiles, int splits, int jobs, cudaStream_t s) {
   if (a.ntile < 16 || a.ntile > kTcMaxTok || a.ntile % 16 != 0) return cudaErrorInvalidValue;
   if (a.ks_len <= 0 || a.ks_len % tc_k_tile(a.fmt) != 0) return cudaErrorInvalidValue;
-  const dim3 grid(row_tiles, a.token_tiles * splits, jobs);
+  const dim3 grid(row_tiles, jobs, a.token_tiles * splits);
   if (a.fmt == FMT_INT4_G32)
     return a.mode == TC_GATEUP ? launch_t<FMT_INT4_G32, TC_GATEUP>(a, grid, s) : launch_t<FMT_INT4_G32, TC_DOWN>(a, grid, s);
   if (a.fmt == FMT_Q4K)

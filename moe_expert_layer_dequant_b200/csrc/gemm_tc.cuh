@@ -42,7 +42,7 @@ struct TcGemmArgs {
   float* out_d;                // DOWN: [splits][slots][N] fp32
   float* out_d_s;              // [splits][M][N]
   int ks_len;                  // K per split (multiple of the weight stage K)
-  int token_tiles;             // grid.y = token_tiles * splits
+  int token_tiles;             // grid.z = token_tiles * splits (token tile major)
 };
 
 // K covered by one weight stage: 256 codes (INT4, Q4_K) or 128 (INT8).

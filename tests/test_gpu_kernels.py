@@ -178,7 +178,7 @@ DENSE_TC = [
 
 
 @pytest.mark.parametrize("cfg,shape", DENSE_TC)
-@pytest.mark.parametrize("M", [3, 16, 40, 150, 300])
+@pytest.mark.parametrize("M", [3, 16, 40, 64, 100, 150, 300])
 def test_dense_tensor_core(cfg, shape, M):
     c = synth.scaled_config(cfg, **shape)
     inp = synth.make_inputs(c, M, 7)
