@@ -23,8 +23,8 @@
  *    never frees them and keeps none after the call returns (plans excepted:
  *    a plan keeps the expert weight pointers until moe_plan_destroy).
  *  - Activations are bf16 (uint16 bit patterns), token-major [M][H], rows
- *    contiguous. x must not alias the output (the pages: the normed input
- *    "must not be the destination of anything encoded in between").
+ *    contiguous. x must not alias the output (on the pages the normed input
+ *    may not be written by any dispatch encoded between its norm and its use).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream) and never synchronize the host. No call reads results
  *    back to the host (the reference's blocking router readback is not
@@ -34,7 +34,8 @@
  *    queries). Its contents need no initialisation and are garbage after.
  *  - Arguments are validated on the host before any launch. Unsupported
  *    combinations are refused with MOEFFN_ERR_UNSUPPORTED and a message; there
- *    is no fallback path (the pages' "refuse rather than degrade").
+ *    is no fallback path (the pages refuse unsupported inputs rather than run
+ *    a lesser path).
  *  - On error the return value is negative and moeffn_last_error() gives a
  *    thread-local message. CUDA launch errors map to MOEFFN_ERR_CUDA.
  *
@@ -132,8 +133,8 @@ int ffn_dense(const moeffn_ffn* w, const uint16_t* x, uint16_t* residual, int M,
  *   m = bf16(x / sqrt(mean(x^2) + eps) * norm_w)   (fp32, over the H columns)
  *   residual[t] = bf16(residual[t] + bf16(down(bf16(act(gate m_t) * (up m_t)))))
  * with x = residual (read before it is updated). turbospark-runtime 0.3.0,
- * src/families/llama/dense.rs, module doc formula box
- * ("m = rms_norm(x, post_attention_layernorm)", there encoded by the caller)
+ * src/families/llama/dense.rs, module doc formula box (the input norm
+ * m = rms_norm(x, post_attention_layernorm), there encoded by the caller)
  * and encode_llama_layer_dense; the norm is the one the pages encode as
  * encode_rms_norm_bf16w. norm_w: [H] bf16, 16-byte aligned; eps >= 0.
  * Few token rows: the norm runs inside the gate/up kernel's staging of the
@@ -225,9 +226,9 @@ size_t moe_workspace_bytes(const moeffn_moe_plan* plan, int M);
  * seed = bf16(bf16(shared(x_t)) * sigmoid(shared_gate . x_t)), or 0.
  * Gemma form (shared_post_norm given): seed = 0 and
  *   residual[t] = bf16(residual[t] + bf16(y[t] + h1[t])), h1 the normed shared branch.
- * turbospark-runtime 0.3.0, src/families/qwen/moe_batch.rs, module doc ("this
- * family's phase 2 SEEDS its accumulator with the gated shared-expert output",
- * "NO SANDWICH NORMS") and encode_qwen_layer_moe_batched.
+ * turbospark-runtime 0.3.0, src/families/qwen/moe_batch.rs, module doc (phase 2
+ * starts its accumulator from the gated shared-expert output; the tail has no
+ * sandwich norm) and encode_qwen_layer_moe_batched.
  * topk_idx_out: optional [M][k] int32 copy of the selected experts. */
 int moe_layer(moeffn_moe_plan* plan, const uint16_t* x, uint16_t* residual, int M, int32_t* topk_idx_out,
               void* ws, size_t ws_bytes, moeffn_stream_t stream);
@@ -239,6 +240,66 @@ int moe_layer(moeffn_moe_plan* plan, const uint16_t* x, uint16_t* residual, int 
  * ffn_dense_prenorm and moe_layer. norm_w: [H] bf16, 16-byte aligned. */
 int moe_layer_prenorm(moeffn_moe_plan* plan, const uint16_t* norm_w, float eps, uint16_t* residual, int M,
                       int32_t* topk_idx_out, void* ws, size_t ws_bytes, moeffn_stream_t stream);
+
+/* ---- Expert-parallel MoE: the routed layer split at its exchange points ----
+ * The batched pass of turbospark-runtime 0.3.0, src/families/qwen/moe_batch.rs
+ * (encode_qwen_layer_moe_batched) groups the (token, rank) pairs by expert,
+ * runs phase 1 (gate/up + activation) and phase 2 (down) per expert of the
+ * union, and sums the expert outputs onto the gated shared-expert seed in rank
+ * order. With the experts spread over GPUs (a contiguous block of E / world
+ * experts per rank), each pair's token row goes to its expert's GPU after the
+ * grouping and its down output comes back before the sum. The three calls
+ * below are the GPU work between those two exchanges, which are the caller's
+ * (e.g. NCCL all-to-alls); the result equals moe_layer's up to the fp32
+ * summation order of the down projection's K splits. The Gemma form is not
+ * covered. */
+
+/* Dispatch order: rows_out[s] = x[perm[s] / top_k], expert_out[s] =
+ * topk_idx[perm[s]] for the M*top_k pair slots s, with topk_idx and perm as
+ * moe_router_topk writes them (pairs in expert order, so each owning rank's
+ * pairs are one contiguous block, of expert_offsets[(r+1)*E/world] -
+ * expert_offsets[r*E/world] rows). x: [M][H] bf16, 16-byte aligned;
+ * topk_idx, perm: [M*top_k] int32; rows_out: [M*top_k][H] bf16, 16-byte
+ * aligned; expert_out: [M*top_k] int32. H a multiple of 8. */
+int moe_dispatch_rows(const uint16_t* x, const int32_t* topk_idx, const int32_t* perm, int M, int top_k, int H,
+                      uint16_t* rows_out, int32_t* expert_out, moeffn_stream_t stream);
+
+/* Workspace bytes of moe_experts_grouped for R rows on this plan (0 if invalid). */
+size_t moe_experts_workspace_bytes(const moeffn_moe_plan* plan, int R);
+
+/* Phases 1 and 2 of the plan's experts over R rows given in any order (as
+ * they arrived from the ranks): d_out[i] = down_e(bf16(act(gate_e . rows[i]) *
+ * (up_e . rows[i]))) in fp32, the down projection's K splits summed in split
+ * order, with e = row_expert[i] - expert_base; a row whose e is outside
+ * [0, E) gives a zero row. The rows are grouped by expert on the device (a
+ * stable counting sort), then run as moe_layer's grouped GEMV or tensor-core
+ * GEMM over the union of experts present. A plan holding one rank's block
+ * of experts (router and top_k unused here; its shared expert is not run)
+ * does exactly that rank's expert work; a plan holding only a shared expert
+ * gives its down output with row_expert all zero. rows: [R][H] bf16;
+ * row_expert: [R] int32; d_out: [R][H] fp32; rows and d_out 16-byte aligned;
+ * at most 1024 experts per plan. R = 0 returns at once. */
+int moe_experts_grouped(moeffn_moe_plan* plan, const uint16_t* rows, int R, const int32_t* row_expert,
+                        int expert_base, float* d_out, void* ws, size_t ws_bytes, moeffn_stream_t stream);
+
+/* Workspace bytes of moe_combine (the inverse of perm). */
+size_t moe_combine_workspace_bytes(int M, int top_k);
+
+/* moe_layer's seeded rank-ordered sum and raw residual add, from the expert
+ * outputs of every pair:
+ *   y[t] = bf16( ((seed[t] + w_0 d_{t,0}) + w_1 d_{t,1}) + ... )  (fp32, rank order)
+ *   residual[t] = bf16(residual[t] + y[t])
+ * with d_{t,r} the row of d at the slot s where perm[s] = t*top_k + r, w =
+ * topk_w, seed[t] = bf16(bf16(shared_d[t]) * sigmoid(gate_logit[t])), or 0
+ * when shared_d is null. d: [M*top_k][H] fp32 in perm's slot order (as
+ * moe_dispatch_rows sent the rows); perm: [M*top_k] int32; topk_w: [M][top_k]
+ * fp32; shared_d: [M][H] fp32 (moe_experts_grouped on a shared-expert plan) or
+ * null; gate_logit: [M] fp32 (moe_router_topk's logits with the shared gate
+ * vector as a one-row router), required with shared_d; residual: [M][H] bf16,
+ * updated in place. d, shared_d, residual 16-byte aligned; H a multiple of 4. */
+int moe_combine(const float* d, const int32_t* perm, const float* topk_w, int M, int top_k, int H,
+                const float* shared_d, const float* gate_logit, uint16_t* residual, void* ws, size_t ws_bytes,
+                moeffn_stream_t stream);
 
 /* Failure detection. Pipeline waits inside the kernels are bounded (about one
  * second); a wait that runs out sets a bit in a device fault word and the

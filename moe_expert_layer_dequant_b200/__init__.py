@@ -84,6 +84,11 @@ _SIGS = {
     "moeffn_profile_read": (_i, [ctypes.c_char_p, _i, _vp, _vp, _i, ctypes.POINTER(_i)]),
     "moeffn_test_topk_from_logits": (_i, [_vp, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moeffn_test_inject_gemv_fault": (_i, [_i, _i, ctypes.c_uint]),
+    "moe_dispatch_rows": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp]),
+    "moe_experts_workspace_bytes": (_sz, [_vp, _i]),
+    "moe_experts_grouped": (_i, [_vp, _vp, _i, _vp, _i, _vp, _vp, _sz, _vp]),
+    "moe_combine_workspace_bytes": (_sz, [_i, _i]),
+    "moe_combine": (_i, [_vp, _vp, _vp, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -407,3 +412,45 @@ def test_topk_from_logits(logits: torch.Tensor, top_k: int, stream=None):
 __all__ = ["ffn_dense", "ffn_dense_prenorm", "moe_layer_prenorm", "ffn_dense_noalloc", "ffn_shared_expert", "moe_router_topk", "moe_layer", "MoePlan", "QWeight", "FFN",
            "qweight_from_arrays", "upload_qweight", "upload_ffn", "plain_weight", "workspace_bytes", "alloc_workspace", "test_dequant",
            "test_topk_from_logits", "test_inject_gemv_fault", "profile_enable", "profile_read", "device_faults", "MoeffnError", "LIB_PATH"]
+
+
+# ----------------------------------------------------------------------------- expert-parallel pieces
+
+
+def moe_dispatch_rows(x: torch.Tensor, topk_idx: torch.Tensor, perm: torch.Tensor, top_k: int, stream=None):
+    """Token rows of the M*k pair slots in perm's (expert) order and each slot's
+    expert: returns (rows bf16 bits [M*k][H], experts int32 [M*k])."""
+    M, H = x.shape
+    P = M * top_k
+    rows = torch.empty((P, H), dtype=x.dtype, device=x.device)
+    experts = torch.empty(P, dtype=torch.int32, device=x.device)
+    _check(_lib.moe_dispatch_rows(_ptr(x), _ptr(topk_idx), _ptr(perm), M, top_k, H, _ptr(rows), _ptr(experts),
+                                  _stream(stream)))
+    return rows, experts
+
+
+def moe_experts_grouped(plan: MoePlan, rows: torch.Tensor, row_expert: torch.Tensor, expert_base: int = 0,
+                        d_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Down outputs (fp32 [R][H]) of the plan's experts for rows in any order:
+    row i goes through expert row_expert[i] - expert_base of the plan."""
+    R, H = rows.shape
+    if d_out is None:
+        d_out = torch.empty((R, H), dtype=torch.float32, device=rows.device)
+    if R == 0:
+        return d_out
+    ws, wp, wn = _ws(ws, lambda: int(_lib.moe_experts_workspace_bytes(plan._h, R)))
+    _check(_lib.moe_experts_grouped(plan._h, _ptr(rows), R, _ptr(row_expert), int(expert_base), _ptr(d_out), wp, wn,
+                                    _stream(stream)))
+    return d_out
+
+
+def moe_combine(d: torch.Tensor, perm: torch.Tensor, topk_w: torch.Tensor, residual: torch.Tensor,
+                shared_d: Optional[torch.Tensor] = None, gate_logit: Optional[torch.Tensor] = None,
+                ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """residual <- bf16(residual + bf16(seed + sum_r w_r d_{t,r})), d in perm's slot order (fp32 [M*k][H])."""
+    M, H = residual.shape
+    k = topk_w.shape[1]
+    ws, wp, wn = _ws(ws, lambda: int(_lib.moe_combine_workspace_bytes(M, k)))
+    _check(_lib.moe_combine(_ptr(d), _ptr(perm), _ptr(topk_w), M, k, H, _ptr(shared_d), _ptr(gate_logit),
+                            _ptr(residual), wp, wn, _stream(stream)))
+    return residual

@@ -9,6 +9,7 @@
 
 #include "../../include/moeffn.h"
 #include "common.cuh"
+#include "ep.cuh"
 #include "gemm_tc.cuh"
 #include "gemv_tma.cuh"
 #include "tmap.cuh"
@@ -842,74 +843,17 @@ size_t moe_workspace_bytes(const moeffn_moe_plan* p, int M) {
 
 namespace {
 
-// moe_layer and moe_layer_prenorm: with norm_w, x is null and the input is
-// m = rms_norm(residual, norm_w), formed by the router kernel.
-int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint16_t* norm_w, float eps,
-              uint16_t* residual, int M, int32_t* topk_idx_out, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
-  g_last_error.clear();
-  if (p == nullptr || residual == nullptr || (x == nullptr && norm_w == nullptr))
-    return fail(MOEFFN_ERR_INVALID, "%s: null pointer", who);
-  if (M < 1) return fail(MOEFFN_ERR_INVALID, "%s: M=%d", who, M);
-  if (norm_w != nullptr) {
-    if (!aligned16(norm_w)) return fail(MOEFFN_ERR_INVALID, "%s: norm weight not 16-byte aligned", who);
-    if (!(eps >= 0.0f)) return fail(MOEFFN_ERR_INVALID, "%s: eps must be >= 0", who);
-  }
-  if ((x != nullptr && !aligned16(x)) || !aligned16(residual))
-    return fail(MOEFFN_ERR_INVALID, "%s: x/residual not 16-byte aligned", who);
-  if (x == residual) return fail(MOEFFN_ERR_INVALID, "%s: x aliases residual", who);
-  const int E = p->E, k = p->k, H = p->H, Ie = p->Ie, Is = p->Is;
-  Carve c{nullptr};
-  carve_moe(c, M, H, Ie, Is, E, k);
-  int rc = check_ws(ws, ws_bytes, c.off);
-  if (rc != MOEFFN_OK) return rc;
-  Carve cw{static_cast<char*>(ws)};
-  const MoeWS w = carve_moe(cw, M, H, Ie, Is, E, k);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+// Phase 1 (grouped gate/up + activation) and phase 2 (grouped down into the
+// fp32 K-split partials w.d, w.d_s) over the pairs grouped in w (perm, offsets,
+// union_list, n_union): pair slot i reads token row perm[i] / k of x. With
+// use_shared the plan's shared expert runs as one more job over all M rows.
+// The split counts of w.d and w.d_s go to *splits_r_out and *splits_s_out.
+int run_moe_phases(moeffn_moe_plan* p, const uint16_t* x, int M, int k, const MoeWS& w, bool use_shared,
+                   cudaStream_t s, int* splits_r_out, int* splits_s_out) {
+  const int E = p->E, H = p->H, Ie = p->Ie, Is = p->Is;
   const int P = M * k;
-
-  RouterArgs ra{};
-  ra.router = p->router;
-  ra.router_f32 = p->router_fmt == MOEFFN_F32;
-  ra.w_sg = p->has_shared ? p->w_sg : nullptr;   // null in the Gemma form (no gate)
-  ra.x = norm_w != nullptr ? residual : x;
-  ra.M = M;
-  ra.H = H;
-  ra.E = E;
-  ra.logits = w.logits;
-  ra.gate_logit = w.gate_logit;
-  ra.route_cnt = w.route_cnt;
-  if (norm_w != nullptr) {   // the router kernel forms m for every later step
-    ra.norm_w = norm_w;
-    ra.eps = eps;
-    ra.m_out = w.m;
-    x = w.m;
-  }
-  {
-    ProfScope ps("router_logits", s);
-    MOEFFN_CHECK_CUDA(launch_router_logits(ra, s), "router launch");
-  }
-
-  RouteArgs rt{};
-  rt.logits = w.logits;
-  rt.M = M;
-  rt.E = E;
-  rt.k = k;
-  rt.idx = topk_idx_out != nullptr ? topk_idx_out : w.idx;
-  rt.w = w.w;
-  rt.perm = w.perm;
-  rt.inv = w.inv;
-  rt.offsets = w.offsets;
-  rt.union_list = w.union_list;
-  rt.n_union = w.n_union;
-  rt.scale = p->expert_scale;
-  rt.counter = w.route_cnt;
-  {
-    ProfScope ps("route_topk", s);
-    MOEFFN_CHECK_CUDA(launch_route(rt, s), "route launch");
-  }
-
   const int routed_jobs = std::min(E, P);
-  const int jobs = routed_jobs + (p->has_shared ? 1 : 0);
+  const int jobs = routed_jobs + (use_shared ? 1 : 0);
   const int max_tok = M;  // a token selects an expert at most once
   const MoeSplit sp = moe_split(Ie, Is);
   const int splits_r = sp.routed, splits_sh = sp.shared;
@@ -1008,7 +952,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     g.act = p->act;
     g.tab0 = p->d_gate;
     g.tab1 = p->d_up;
-    if (p->has_shared) {
+    if (use_shared) {
       g.s0 = to_qw(p->shared.gate);
       g.s1 = to_qw(p->shared.up);
       g.Ns = Is;
@@ -1040,7 +984,7 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     TmaGemvArgs d{};
     d.fmt = MOEFFN_Q_INT4_AFFINE_G32;
     d.tab0 = p->d_down;
-    if (p->has_shared) {
+    if (use_shared) {
       d.s0 = to_qw(p->shared.down);
       d.Ns = H;
       d.Ks = Is;
@@ -1072,6 +1016,79 @@ int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint
     }
   }
 
+  *splits_r_out = tc_splits_r;
+  *splits_s_out = tc_splits_s;
+  return MOEFFN_OK;
+}
+
+// moe_layer and moe_layer_prenorm: with norm_w, x is null and the input is
+// m = rms_norm(residual, norm_w), formed by the router kernel.
+int moe_entry(const char* who, moeffn_moe_plan* p, const uint16_t* x, const uint16_t* norm_w, float eps,
+              uint16_t* residual, int M, int32_t* topk_idx_out, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
+  g_last_error.clear();
+  if (p == nullptr || residual == nullptr || (x == nullptr && norm_w == nullptr))
+    return fail(MOEFFN_ERR_INVALID, "%s: null pointer", who);
+  if (M < 1) return fail(MOEFFN_ERR_INVALID, "%s: M=%d", who, M);
+  if (norm_w != nullptr) {
+    if (!aligned16(norm_w)) return fail(MOEFFN_ERR_INVALID, "%s: norm weight not 16-byte aligned", who);
+    if (!(eps >= 0.0f)) return fail(MOEFFN_ERR_INVALID, "%s: eps must be >= 0", who);
+  }
+  if ((x != nullptr && !aligned16(x)) || !aligned16(residual))
+    return fail(MOEFFN_ERR_INVALID, "%s: x/residual not 16-byte aligned", who);
+  if (x == residual) return fail(MOEFFN_ERR_INVALID, "%s: x aliases residual", who);
+  const int E = p->E, k = p->k, H = p->H, Ie = p->Ie, Is = p->Is;
+  Carve c{nullptr};
+  carve_moe(c, M, H, Ie, Is, E, k);
+  int rc = check_ws(ws, ws_bytes, c.off);
+  if (rc != MOEFFN_OK) return rc;
+  Carve cw{static_cast<char*>(ws)};
+  const MoeWS w = carve_moe(cw, M, H, Ie, Is, E, k);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int P = M * k;
+
+  RouterArgs ra{};
+  ra.router = p->router;
+  ra.router_f32 = p->router_fmt == MOEFFN_F32;
+  ra.w_sg = p->has_shared ? p->w_sg : nullptr;   // null in the Gemma form (no gate)
+  ra.x = norm_w != nullptr ? residual : x;
+  ra.M = M;
+  ra.H = H;
+  ra.E = E;
+  ra.logits = w.logits;
+  ra.gate_logit = w.gate_logit;
+  ra.route_cnt = w.route_cnt;
+  if (norm_w != nullptr) {   // the router kernel forms m for every later step
+    ra.norm_w = norm_w;
+    ra.eps = eps;
+    ra.m_out = w.m;
+    x = w.m;
+  }
+  {
+    ProfScope ps("router_logits", s);
+    MOEFFN_CHECK_CUDA(launch_router_logits(ra, s), "router launch");
+  }
+
+  RouteArgs rt{};
+  rt.logits = w.logits;
+  rt.M = M;
+  rt.E = E;
+  rt.k = k;
+  rt.idx = topk_idx_out != nullptr ? topk_idx_out : w.idx;
+  rt.w = w.w;
+  rt.perm = w.perm;
+  rt.inv = w.inv;
+  rt.offsets = w.offsets;
+  rt.union_list = w.union_list;
+  rt.n_union = w.n_union;
+  rt.scale = p->expert_scale;
+  rt.counter = w.route_cnt;
+  {
+    ProfScope ps("route_topk", s);
+    MOEFFN_CHECK_CUDA(launch_route(rt, s), "route launch");
+  }
+
+  int tc_splits_r = 0, tc_splits_s = 0;
+  if ((rc = run_moe_phases(p, x, M, k, w, p->has_shared, s, &tc_splits_r, &tc_splits_s)) != MOEFFN_OK) return rc;
   TailArgs t{};
   t.mode = p->shared_post_norm != nullptr ? TAIL_MOE_GEMMA : TAIL_MOE;
   t.norm_w = p->shared_post_norm;
@@ -1107,6 +1124,111 @@ int moe_layer_prenorm(moeffn_moe_plan* p, const uint16_t* norm_w, float eps, uin
                       int32_t* topk_idx_out, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
   if (norm_w == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_layer_prenorm: null norm weight");
   return moe_entry("moe_layer_prenorm", p, nullptr, norm_w, eps, residual, M, topk_idx_out, ws, ws_bytes, stream);
+}
+
+// ---- expert-parallel pieces ------------------------------------------------
+
+int moe_dispatch_rows(const uint16_t* x, const int32_t* topk_idx, const int32_t* perm, int M, int top_k, int H,
+                      uint16_t* rows_out, int32_t* expert_out, moeffn_stream_t stream) {
+  g_last_error.clear();
+  if (x == nullptr || topk_idx == nullptr || perm == nullptr || rows_out == nullptr || expert_out == nullptr)
+    return fail(MOEFFN_ERR_INVALID, "moe_dispatch_rows: null pointer");
+  if (M < 1 || top_k < 1 || top_k > kMaxTopK || H < 8 || H % 8 != 0)
+    return fail(MOEFFN_ERR_INVALID, "moe_dispatch_rows: M=%d top_k=%d H=%d (H a positive multiple of 8)", M, top_k, H);
+  if (!aligned16(x) || !aligned16(rows_out)) return fail(MOEFFN_ERR_INVALID, "moe_dispatch_rows: x/rows_out not 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  DispatchArgs a{x, topk_idx, perm, M * top_k, top_k, H, rows_out, expert_out};
+  ProfScope ps("dispatch_rows", s);
+  MOEFFN_CHECK_CUDA(launch_dispatch_rows(a, s), "dispatch launch");
+  return MOEFFN_OK;
+}
+
+size_t moe_experts_workspace_bytes(const moeffn_moe_plan* p, int R) {
+  if (p == nullptr || R < 1) return 0;
+  Carve c{nullptr};
+  carve_moe(c, R, p->H, p->Ie, p->Is, p->E, 1);
+  return c.off;
+}
+
+int moe_experts_grouped(moeffn_moe_plan* p, const uint16_t* rows, int R, const int32_t* row_expert,
+                        int expert_base, float* d_out, void* ws, size_t ws_bytes, moeffn_stream_t stream) {
+  g_last_error.clear();
+  if (p == nullptr) return fail(MOEFFN_ERR_INVALID, "moe_experts_grouped: null plan");
+  if (R < 0 || expert_base < 0) return fail(MOEFFN_ERR_INVALID, "moe_experts_grouped: R=%d expert_base=%d", R, expert_base);
+  if (R == 0) return MOEFFN_OK;
+  if (rows == nullptr || row_expert == nullptr || d_out == nullptr)
+    return fail(MOEFFN_ERR_INVALID, "moe_experts_grouped: null pointer");
+  if (!aligned16(rows) || !aligned16(d_out))
+    return fail(MOEFFN_ERR_INVALID, "moe_experts_grouped: rows/d_out not 16-byte aligned");
+  if (p->E > kMaxExperts) return fail(MOEFFN_ERR_UNSUPPORTED, "moe_experts_grouped: %d experts (at most %d)", p->E, kMaxExperts);
+  const int E = p->E, H = p->H, Ie = p->Ie, Is = p->Is;
+  Carve c{nullptr};
+  carve_moe(c, R, H, Ie, Is, E, 1);
+  int rc = check_ws(ws, ws_bytes, c.off);
+  if (rc != MOEFFN_OK) return rc;
+  Carve cw{static_cast<char*>(ws)};
+  const MoeWS w = carve_moe(cw, R, H, Ie, Is, E, 1);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  {
+    PlaceArgs pa{row_expert, R, expert_base, E, w.offsets, w.perm, w.inv, w.union_list, w.n_union};
+    ProfScope ps("place_rows", s);
+    MOEFFN_CHECK_CUDA(launch_place_rows(pa, s), "row placement launch");
+  }
+  // Each row is one pair (k = 1): slot i of the grouped order reads row perm[i].
+  int splits_r = 0, splits_s = 0;
+  if ((rc = run_moe_phases(p, rows, R, 1, w, false, s, &splits_r, &splits_s)) != MOEFFN_OK) return rc;
+  RowsFromSlotsArgs ra{w.d, splits_r, R, H, R, w.inv, d_out};
+  ProfScope ps("rows_from_slots", s);
+  MOEFFN_CHECK_CUDA(launch_rows_from_slots(ra, s), "split sum launch");
+  return MOEFFN_OK;
+}
+
+size_t moe_combine_workspace_bytes(int M, int top_k) {
+  if (M < 1 || top_k < 1) return 0;
+  Carve c{nullptr};
+  c.take<int>((size_t)M * top_k);
+  return c.off;
+}
+
+int moe_combine(const float* d, const int32_t* perm, const float* topk_w, int M, int top_k, int H,
+                const float* shared_d, const float* gate_logit, uint16_t* residual, void* ws, size_t ws_bytes,
+                moeffn_stream_t stream) {
+  g_last_error.clear();
+  if (d == nullptr || perm == nullptr || topk_w == nullptr || residual == nullptr)
+    return fail(MOEFFN_ERR_INVALID, "moe_combine: null pointer");
+  if (shared_d != nullptr && gate_logit == nullptr)
+    return fail(MOEFFN_ERR_INVALID, "moe_combine: shared_d needs gate_logit");
+  if (M < 1 || top_k < 1 || top_k > kMaxTopK || H < 4 || H % 4 != 0)
+    return fail(MOEFFN_ERR_INVALID, "moe_combine: M=%d top_k=%d H=%d (H a positive multiple of 4)", M, top_k, H);
+  if (!aligned16(d) || !aligned16(residual) || (shared_d != nullptr && !aligned16(shared_d)))
+    return fail(MOEFFN_ERR_INVALID, "moe_combine: d/shared_d/residual not 16-byte aligned");
+  int rc = check_ws(ws, ws_bytes, moe_combine_workspace_bytes(M, top_k));
+  if (rc != MOEFFN_OK) return rc;
+  Carve cw{static_cast<char*>(ws)};
+  int* inv = cw.take<int>((size_t)M * top_k);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  {
+    InvertArgs ia{perm, M * top_k, inv};
+    ProfScope ps("invert_perm", s);
+    MOEFFN_CHECK_CUDA(launch_invert_perm(ia, s), "permutation inverse launch");
+  }
+  TailArgs t{};
+  t.mode = TAIL_MOE;
+  t.M = M;
+  t.N = H;
+  t.d = d;
+  t.splits = 1;
+  t.slots = M * top_k;
+  t.d_s = shared_d;
+  t.splits_s = shared_d != nullptr ? 1 : 0;
+  t.gate_logit = gate_logit;
+  t.w = topk_w;
+  t.inv = inv;
+  t.k = top_k;
+  t.res = residual;
+  ProfScope ps("tail_moe", s);
+  MOEFFN_CHECK_CUDA(launch_tail(t, s), "moe tail launch");
+  return MOEFFN_OK;
 }
 
 }  // extern "C"
