@@ -251,7 +251,7 @@ def ffn_hidden(weights, x: np.ndarray, act: str) -> np.ndarray:
 
 def residual_add(res: np.ndarray, y_bf16: np.ndarray) -> np.ndarray:
     """x = x + h: ``encode_residual_add`` of a bf16 row into the bf16 stream.
-    The only tail of the llama layer ([llama], "RAW residual add")."""
+    The only tail of the llama layer ([llama]: a plain residual add, no norm)."""
     return bf16(res + y_bf16)
 
 
@@ -374,8 +374,8 @@ def shared_seed(shared, w_sg_bits: np.ndarray, x_bits: np.ndarray, act: str) -> 
 def seeded_rank_sum(seed: np.ndarray, w: np.ndarray, d: np.ndarray) -> np.ndarray:
     """y = bf16(((seed + w0 d0) + w1 d1) + ...) with an fp32 accumulator.
 
-    [qwen] phase-2 call: the kernel "starts its accumulator at the gated shared
-    expert and then adds the eight ranks" -- the seed is the start, not a later
+    [qwen] phase-2 call: the kernel's accumulator begins at the gated shared
+    expert and the ranks are added after it in order -- the seed is the start, not a later
     addend. seed [M][H], w [M][k], d [M][k][H] (d rounded to fp32 here).
     """
     acc = f32(seed)
