@@ -135,6 +135,11 @@ class ExpertParallelMoE:
 
     # -- the three local steps ------------------------------------------------
     def begin(self, x: torch.Tensor) -> Pending:
+        if x.shape[0] == 0:
+            # No token rows here: nothing to send, but this rank still takes
+            # every collective step (and holds experts for the others' rows).
+            return Pending(None, None, x.new_empty((0,) + tuple(x.shape[1:])),
+                           torch.empty(0, dtype=torch.int32, device=x.device), [0] * self.world)
         idx, w, perm, offsets = self.ops.route(x)
         rows, experts = self.ops.dispatch(x, idx, perm)
         send = send_counts(offsets.cpu().tolist(), self.E, self.world)
@@ -144,6 +149,8 @@ class ExpertParallelMoE:
         return self.ops.experts(rows, experts)
 
     def finish(self, p: Pending, d_back, x: torch.Tensor, residual: torch.Tensor) -> torch.Tensor:
+        if residual.shape[0] == 0:
+            return residual
         self.ops.combine(d_back, p.perm, p.w, residual, self.ops.shared(x))
         return residual
 

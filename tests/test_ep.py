@@ -132,3 +132,8 @@ def test_a_rank_that_receives_no_rows():
     # one token row with top-2 of 8 experts reaches at most 2 of 4 ranks; the
     # others exchange empty blocks and still take every collective step
     _spawn(4, "mixtral", [1, 1, 1, 1])
+
+
+def test_a_rank_without_token_rows():
+    # rank 1 routes nothing but holds experts for rank 0's rows
+    _spawn(2, "qwen", [6, 0])
