@@ -142,7 +142,9 @@ class ExpertParallelMoE:
                            torch.empty(0, dtype=torch.int32, device=x.device), [0] * self.world)
         idx, w, perm, offsets = self.ops.route(x)
         rows, experts = self.ops.dispatch(x, idx, perm)
-        send = send_counts(offsets.cpu().tolist(), self.E, self.world)
+        # The split sizes of the all-to-all are read back to the host (a
+        # synchronization); one rank keeps every row and needs none.
+        send = [rows.shape[0]] if self.world == 1 else send_counts(offsets.cpu().tolist(), self.E, self.world)
         return Pending(w, perm, rows, experts, send)
 
     def expert_work(self, rows: torch.Tensor, experts: torch.Tensor):
