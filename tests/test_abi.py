@@ -150,3 +150,31 @@ def test_fault_injection_export_validates_on_the_host():
             lib.test_inject_gemv_fault(*args)
         assert e.value.status == -1
     lib.test_inject_gemv_fault(0)                  # cancel: always accepted
+
+
+@nogpu
+def test_expert_parallel_refusals():
+    """moe_dispatch_rows, moe_experts_grouped and moe_combine validate on the
+    host before any launch; workspace queries size the combine's inverse map."""
+    import moe_expert_layer_dequant_b200 as lib
+    L = lib._lib
+    x, idx, perm, rows, exp = 0x40000000, 0x41000000, 0x42000000, 0x43000000, 0x44000000
+    assert L.moe_dispatch_rows(None, idx, perm, 4, 2, 256, rows, exp, None) == -1
+    assert L.moe_dispatch_rows(x, idx, perm, 0, 2, 256, rows, exp, None) == -1       # M = 0
+    assert L.moe_dispatch_rows(x, idx, perm, 4, 0, 256, rows, exp, None) == -1       # top_k = 0
+    assert L.moe_dispatch_rows(x, idx, perm, 4, 17, 256, rows, exp, None) == -1      # top_k above 16
+    assert L.moe_dispatch_rows(x, idx, perm, 4, 2, 260, rows, exp, None) == -1       # H % 8 != 0
+    assert L.moe_dispatch_rows(x + 2, idx, perm, 4, 2, 256, rows, exp, None) == -1   # misaligned x
+    assert b"aligned" in L.moeffn_last_error()
+    assert L.moe_experts_grouped(None, rows, 8, exp, 0, 0x45000000, 0x60000000, 1 << 20, None) == -1
+    assert L.moe_experts_workspace_bytes(None, 8) == 0
+    d, w, res, sd, ws = 0x46000000, 0x47000000, 0x48000000, 0x49000000, 0x60000000
+    need = L.moe_combine_workspace_bytes(4, 2)
+    assert need >= 4 * 2 * 4 and L.moe_combine_workspace_bytes(0, 2) == 0
+    assert L.moe_combine(None, perm, w, 4, 2, 256, None, None, res, ws, need, None) == -1
+    assert L.moe_combine(d, perm, w, 4, 2, 256, sd, None, res, ws, need, None) == -1   # shared_d without its gate
+    assert b"gate_logit" in L.moeffn_last_error()
+    assert L.moe_combine(d, perm, w, 0, 2, 256, None, None, res, ws, need, None) == -1  # M = 0
+    assert L.moe_combine(d, perm, w, 4, 2, 258, None, None, res, ws, need, None) == -1  # H % 4 != 0
+    assert L.moe_combine(d + 4, perm, w, 4, 2, 256, None, None, res, ws, need, None) == -1
+    assert L.moe_combine(d, perm, w, 4, 2, 256, None, None, res, ws, need - 1, None) == -3
