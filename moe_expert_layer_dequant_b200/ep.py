@@ -66,6 +66,7 @@ class GpuOps:
         # The shared expert as a one-expert plan whose router row is the gate
         # vector: its logits are the gate logits, its expert output the seed's s.
         self.shared_plan = None
+        self._zero_ids = {}   # row count -> int32 zeros: the shared plan's expert of every row
         if shared is not None:
             if shared_gate is None:
                 raise ValueError("a shared expert needs its gate vector")
@@ -91,7 +92,9 @@ class GpuOps:
         M = x.shape[0]
         z = torch.empty((M, 1), dtype=torch.float32, device=x.device)
         moe_router_topk(self.shared_plan.router, x, 1, logits_out=z)
-        zeros = torch.zeros(M, dtype=torch.int32, device=x.device)
+        zeros = self._zero_ids.get(M)
+        if zeros is None or zeros.device != x.device:
+            zeros = self._zero_ids[M] = torch.zeros(M, dtype=torch.int32, device=x.device)
         s = moe_experts_grouped(self.shared_plan, x, zeros, 0)
         return s, z.reshape(M)
 
