@@ -137,3 +137,64 @@ def test_a_rank_that_receives_no_rows():
 def test_a_rank_without_token_rows():
     # rank 1 routes nothing but holds experts for rank 0's rows
     _spawn(2, "qwen", [6, 0])
+
+
+# --------------------------------------------------------------------------- hand-derived layers
+
+
+GOLDEN = {
+    # builder, golden fixture, key of the expected output at feature 0 (per token row)
+    "rank_pairing": ("rank_pairing_layer", "rank_weight_pairing.txt", "y_feature0"),
+    "shared_gate": ("shared_gate_layer", "shared_gate_seed.txt", "seed_feature0"),
+    "seed_first": ("seed_counterexample", None, None),          # y = 0 exactly (seed, then the ranks)
+}
+
+
+def _golden_rank_main(rank, world, port, name, out):
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    import handbuilt
+    from ep_oracle_ops import OracleOps
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        li = getattr(handbuilt, GOLDEN[name][0])(32, 1)
+        tokens = [t for t in range(li.x.shape[0]) if t % world == rank]
+        x = torch.from_numpy(li.x[tokens].view(np.int16).copy())
+        res = torch.from_numpy(li.residual[tokens].view(np.int16).copy())
+        ExpertParallelMoE(OracleOps(li, rank, world), li.config.E, group=dist.group.WORLD).forward(x, res)
+        out.put((rank, tokens, res.numpy().view(np.uint16).copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("name", sorted(GOLDEN))
+def test_hand_derived_layers_with_one_expert_per_rank(name):
+    """The worked examples of tests/golden with each of the two experts on
+    its own rank and the token rows split between the ranks: the pairs cross
+    the exchange and the outputs keep their hand-derived values."""
+    import handbuilt
+    from conftest import read_golden
+    li = getattr(handbuilt, GOLDEN[name][0])(32, 1)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_golden_rank_main, args=(r, 2, port, name, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(240)
+        assert p.exitcode == 0
+    got = np.zeros_like(li.x)
+    for _ in range(2):
+        _, tokens, rows = q.get(timeout=10)
+        got[tokens] = rows
+    _, fixture, key = GOLDEN[name]
+    if fixture is None:
+        want0 = np.zeros(li.x.shape[0])
+    else:
+        kv, _ = read_golden(fixture)
+        want0 = np.array([float(v) for v in kv[key]])
+    assert np.array_equal(oracle.bf16_to_f64(got)[:, 0], want0)
+    assert np.array_equal(got, oracle.layer(li))
