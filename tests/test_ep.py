@@ -29,6 +29,10 @@ SHAPES = {
     "qwen": dict(cfg=4, H=128, I=64, E=8, k=4, I_s=64),
     # Mixtral form: no shared expert, bf16 router, top-2 of 8
     "mixtral": dict(cfg=5, H=128, I=96, E=8, k=2, I_s=0),
+    # top-1 routing (one pair per token)
+    "top1": dict(cfg=5, H=96, I=64, E=4, k=1, I_s=0),
+    # 16 experts, top-4, shared expert: four experts per rank at world 4
+    "wide": dict(cfg=4, H=64, I=32, E=16, k=4, I_s=32),
 }
 
 
@@ -132,6 +136,12 @@ def test_a_rank_that_receives_no_rows():
     # one token row with top-2 of 8 experts reaches at most 2 of 4 ranks; the
     # others exchange empty blocks and still take every collective step
     _spawn(4, "mixtral", [1, 1, 1, 1])
+
+
+@pytest.mark.parametrize("name,world,M_per_rank", [("top1", 2, [4, 7]), ("top1", 4, [2, 2, 2, 2]),
+                                                   ("wide", 4, [5, 1, 3, 6]), ("wide", 2, [9, 2])])
+def test_routing_widths_and_world_sizes(name, world, M_per_rank):
+    _spawn(world, name, M_per_rank)
 
 
 def test_a_rank_without_token_rows():
